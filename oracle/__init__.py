@@ -1,0 +1,27 @@
+"""CPU oracle of gated delta-rule decode over a slot or paged state pool.
+
+TEST INFRASTRUCTURE, NOT PRODUCT CODE. Only the tests, the smoke check of
+``__graft_entry__`` and the CPU-baseline leg of ``bench.py`` may import it.
+The CUDA library never calls it and shares no code with it: the two meet
+only through the seeded input generators in ``workloads``.
+
+The oracle computes in float64 (the fp8 tile codec in binary32, so that
+codes and scales are exactly reproducible) and follows the pages' literal
+step order; see ``oracle.gdn`` for the sources and for every reading of a
+point the pages leave open.
+
+Parity status of each function:
+
+* ``gated_delta_step`` and the pool drivers: pinned by closed forms
+  (alpha=1/beta=0 keeps S; alpha=0/beta=1 gives k v^T; unit-norm key with
+  beta=1 overwrites; beta=0 gives the product of decays), an independent
+  transition-matrix formulation, exact rational arithmetic on tiny inputs,
+  sequential == repeated single steps, and the paged and slot pool rules.
+* ``formats``: pinned by the OCP E4M3 format's defined points, by library
+  conversions (torch bf16 and float8_e4m3fn casts) and by grid properties.
+* conventions the pages do not fix (parity unpinned): the L2-norm epsilon,
+  the GQA head map ``hv // (HV // H)``, the KDA gate's use of the GDN form
+  per key channel, and the tile codec's scale formula.
+"""
+
+from . import formats, gdn  # noqa: F401

@@ -1,0 +1,111 @@
+"""Plant plausible mistakes in the oracle (on the CPU) and check that the pins
+catch every one of them: a pin set that a dropped term, a wrong sign, a
+swapped index or a transposed operand slips through would not be a pin."""
+
+import math
+
+import numpy as np
+import pytest
+
+from oracle import formats
+from oracle import gdn as O
+from pins import ALL_PINS
+
+
+def _step_readout_before_write(S, q_hat, k_hat, v, alpha, beta):
+    S = O.decay(S, alpha)
+    o = O.readout(S, q_hat)
+    v_old = O.delta_read(S, k_hat)
+    S = O.delta_write(S, k_hat, O.delta_residual(v, v_old, beta))
+    return o, S
+
+
+def _step_read_before_decay(S, q_hat, k_hat, v, alpha, beta):
+    v_old = O.delta_read(S, k_hat)
+    S = O.decay(S, alpha)
+    S = O.delta_write(S, k_hat, O.delta_residual(v, v_old, beta))
+    return O.readout(S, q_hat), S
+
+
+def _resolve_ignoring_new_page(page_indices, page_indptr, last_page_len, bb):
+    last = int(page_indptr[bb + 1]) - 1
+    return int(page_indices[last]), int(page_indices[last])
+
+
+def _resolve_writing_old_page(page_indices, page_indptr, last_page_len, bb):
+    r, w = _ORIG_RESOLVE(page_indices, page_indptr, last_page_len, bb)
+    return r, r
+
+
+_ORIG_RESOLVE = O.resolve_pages
+_ORIG_QUANT_TILE = formats.quantize_tile
+
+
+def _tile_wrong_max(tile):
+    t = np.asarray(tile, np.float32)
+    amax = np.float32(np.max(np.abs(t)))
+    if amax == 0:
+        return np.zeros(t.shape, np.uint8), np.float32(0)
+    s = np.float32(amax / np.float32(256.0))
+    return formats.e4m3_encode((t * (np.float32(1) / s)).astype(np.float32)), s
+
+
+def _e4m3_half_away(x):
+    """Round half away from zero: nudge each value one binary32 ulp outwards."""
+    x = np.asarray(x, np.float32)
+    return _ORIG_E4M3(np.nextafter(x, np.sign(x) * np.inf).astype(np.float32))
+
+
+_ORIG_E4M3 = formats.e4m3_encode
+
+MUTATIONS = {
+    "read_transposed": (O, "delta_read", lambda S, k: S @ k),
+    "residual_sign": (O, "delta_residual", lambda v, v_old, beta: beta * (v_old - np.asarray(v, float))),
+    "residual_no_beta": (O, "delta_residual", lambda v, v_old, beta: np.asarray(v, float) - v_old),
+    "decay_dropped": (O, "decay", lambda S, alpha: S),
+    "decay_value_axis": (O, "decay", lambda S, alpha: S * float(alpha) if np.ndim(alpha) == 0
+                         else S * np.asarray(alpha)[None, :]),
+    "write_transposed": (O, "delta_write", lambda S, k, u: S + np.outer(u, k)),
+    "write_dropped": (O, "delta_write", lambda S, k, u: S),
+    "readout_before_write": (O, "gated_delta_step", _step_readout_before_write),
+    "read_before_decay": (O, "gated_delta_step", _step_read_before_decay),
+    "gqa_modulo": (O, "key_head_of", lambda hv, H, HV: hv % H),
+    "gate_sign": (O, "gdn_alpha", lambda A, a, d: math.exp(min(
+        math.exp(float(A)) * float(O.softplus(float(a) + float(d))), 700.0))),
+    "gate_no_dt_bias": (O, "gdn_alpha", lambda A, a, d: math.exp(-math.exp(float(A)) * float(O.softplus(float(a))))),
+    "kda_gate_no_dt_bias": (O, "kda_alpha", lambda A, g, d: np.exp(-math.exp(float(A)) * O.softplus(np.asarray(g, float)))),
+    "softplus_plain_relu": (O, "softplus", lambda x: np.maximum(np.asarray(x, float), 0.0)),
+    "sigmoid_missing": (O, "sigmoid", lambda x: np.asarray(x, float)),
+    "l2_no_eps_norm_sq": (O, "l2_normalize", lambda x: np.asarray(x, float) / (float(np.sum(np.asarray(x, float) ** 2)) + 1e-6)),
+    "qk_scale_dropped": (O, "prepare_qk", lambda q, k, scale, use=True: (O.l2_normalize(q), O.l2_normalize(k))
+                         if use else (np.asarray(q, float), np.asarray(k, float))),
+    "new_page_ignored": (O, "resolve_pages", _resolve_ignoring_new_page),
+    "write_to_read_page": (O, "resolve_pages", _resolve_writing_old_page),
+    "bf16_truncates": (formats, "f32_to_bf16_bits",
+                       lambda x: (np.ascontiguousarray(np.asarray(x, np.float32)).view(np.uint32) >> 16).astype(np.uint16)),
+    "e4m3_half_away": (formats, "e4m3_encode", _e4m3_half_away),
+    "tile_scale_256": (formats, "quantize_tile", _tile_wrong_max),
+}
+
+
+def _pins_fail():
+    failed = []
+    for pin in ALL_PINS:
+        try:
+            with np.errstate(all="ignore"):
+                pin()
+        except Exception as e:  # an exception from a broken oracle counts as a catch
+            failed.append(pin.__name__)
+    return failed
+
+
+def test_unmutated_oracle_passes_all_pins():
+    assert _pins_fail() == []
+
+
+@pytest.mark.parametrize("name", sorted(MUTATIONS))
+def test_mutation_is_caught(name, monkeypatch):
+    mod, attr, fn = MUTATIONS[name]
+    monkeypatch.setattr(mod, attr, fn)
+    failed = _pins_fail()
+    assert failed, f"planted mistake '{name}' passed every pin"

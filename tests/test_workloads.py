@@ -1,0 +1,63 @@
+"""Host logic of the seeded input generators (CPU only)."""
+
+import numpy as np
+
+import workloads as W
+
+
+def test_paged_table_invariants():
+    w = W.WORKLOADS["paged"]
+    pt = W.paged_table(w.seed, w.B, w.page_size, w.max_len, w.n_share, w.share_pages,
+                       force_lens={0: 1025, 1: 1025})
+    assert pt.page_indptr[0] == 0 and np.all(np.diff(pt.page_indptr) >= 1)
+    assert len(pt.page_indices) == pt.page_indptr[-1]
+    assert np.all((pt.last_page_len >= 1) & (pt.last_page_len <= w.page_size))
+    assert np.all((pt.seq_lens >= 2) & (pt.seq_lens <= w.max_len))
+    npages = np.diff(pt.page_indptr)
+    assert np.array_equal(npages, -(-pt.seq_lens // w.page_size))
+    # sharers start with the same prefix pages and go past it
+    for b in range(w.n_share):
+        row = pt.page_indices[pt.page_indptr[b]:pt.page_indptr[b + 1]]
+        assert np.array_equal(row[:w.share_pages], pt.shared_pages)
+        assert pt.seq_lens[b] > w.share_pages * w.page_size
+    # forced sequences open a new page right after the shared prefix
+    assert pt.last_page_len[0] == 1 and pt.last_page_len[1] == 1
+    # write pages (last page of each sequence) are distinct and never shared
+    last = pt.page_indices[pt.page_indptr[1:] - 1]
+    assert len(set(last.tolist())) == w.B
+    assert not set(last.tolist()) & set(pt.shared_pages.tolist())
+    # every page id is used, only the shared ones more than once
+    ids, counts = np.unique(pt.page_indices, return_counts=True)
+    assert len(ids) == pt.num_pages and ids.max() == pt.num_pages - 1
+    assert set(ids[counts > 1].tolist()) == set(pt.shared_pages.tolist())
+
+
+def test_slot_rotations_disjoint_and_reproducible():
+    sets = [W.slot_indices(1, 64, 256, r) for r in range(4)]
+    allv = np.concatenate(sets)
+    assert len(set(allv.tolist())) == 256
+    assert np.array_equal(sets[0], W.slot_indices(1, 64, 256, 0))
+
+
+def test_varlen_offsets():
+    cu = W.varlen_offsets(3, 32, 8)
+    lens = np.diff(cu)
+    assert cu[0] == 0 and np.all((lens >= 1) & (lens <= 8)) and cu.dtype == np.int32
+
+
+def test_layouts_hold_same_logical_state():
+    a, _ = W.slot_state(3, 5, 2, 8, 4, "K_FIRST", "f32")
+    b, _ = W.slot_state(3, 5, 2, 8, 4, "V_FIRST", "f32")
+    assert np.array_equal(a, b.transpose(0, 2, 1))
+    bits, _ = W.slot_state(3, 5, 2, 8, 4, "V_FIRST", "bf16")
+    assert bits.dtype == np.uint16 and bits.shape == (2, 4, 8)
+    codes, scales = W.slot_state(4, 0, 2, 8, 128, "V_FIRST", "fp8_e4m3", 64)
+    assert codes.dtype == np.uint8 and scales.shape == (2, 2)
+    assert not np.any((codes & 0x7F) == 0x7F)   # no NaN codes
+
+
+def test_bf16_inputs_are_representable():
+    t = W.gdn_tokens(1, 2, 1, 2, 4, 8, 8, "bf16")
+    for n in ("q", "k", "v", "a", "b"):
+        x = t[n].view(np.uint32)
+        assert np.all((x & 0xFFFF) == 0)
