@@ -1,0 +1,327 @@
+// Device helpers shared by the decode kernels: state storage formats, vector
+// loads and stores, the token prologue (activations, norms) and the
+// resolution of a (sequence) unit to its pool slots or pages.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp8.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace gdn {
+
+// ---------------------------------------------------------------------------
+// enums shared with the host side (values match include/gdn.h)
+// ---------------------------------------------------------------------------
+enum StateFmt : int { ST_F32 = 0, ST_BF16 = 1, ST_FP8 = 2 };
+enum Layout : int { L_KFIRST = 0, L_VFIRST = 1 };
+enum IndexMode : int { IDX_SLOTS = 0, IDX_PAGED = 1 };
+enum GateKind : int { GATE_SCALAR = 0, GATE_VECTOR = 1 };
+
+// run-time flags of one call
+constexpr int F_IN_BF16 = 1;
+constexpr int F_OUT_BF16 = 2;
+constexpr int F_IDX64 = 4;
+constexpr int F_L2NORM = 8;
+constexpr int F_BETA_PROB = 16;
+constexpr int F_READOUT_STORED = 32;
+constexpr int F_VARLEN = 64;
+
+// err_flags bits (GDN_FLAG_* in the public header)
+constexpr int E_SLOT_RANGE = 1;
+constexpr int E_PAGE_RANGE = 2;
+constexpr int E_PAGE_TABLE = 4;
+constexpr int E_SEQLENS = 8;
+
+constexpr float kL2Eps = 1e-6f;
+constexpr float kE4M3Max = 448.0f;
+constexpr unsigned kFull = 0xffffffffu;
+
+// Everything one launch needs. Token-major inputs: GDN [B, T, ...] is the
+// token axis tok = b * T + t; KDA uses the varlen token axis directly.
+struct StepParams {
+  const void* q;        // [tok, H, K]
+  const void* k;        // [tok, H, K]
+  const void* v;        // [tok, HV, V]
+  const void* gate;     // GDN a [tok, HV]; KDA raw_gate [tok, HV, K]
+  const void* beta;     // [tok, HV]
+  const float* A_log;   // [HV]
+  const float* dt_bias; // GDN [HV]; KDA [HV, K]
+  void* pool;           // [num_slots, HV, state]
+  float* scales;        // fp8: [num_slots, HV, V / 64]
+  const void* idx;      // slots: state_indices [B]; paged: page_indices [nnz]
+  const void* indptr;   // paged: page_indptr [B+1]; varlen: cu_seqlens [B+1] int32
+  const void* lastlen;  // paged: last_page_len [B]
+  const int64_t* rows;  // paged: precomputed (read, write) [B, 2] or null
+  void* out;            // [tok, HV, V]
+  int32_t* err;         // optional
+  int64_t num_slots;
+  int64_t nnz;
+  int B, T, H, HV, V;
+  int n_vtiles;
+  int total_tokens;
+  int page_size;
+  float scale;
+  int flags;
+};
+
+// ---------------------------------------------------------------------------
+// state formats: 16 bytes hold EPL elements
+// ---------------------------------------------------------------------------
+template <int SDT> struct StateTraits;
+template <> struct StateTraits<ST_F32> { static constexpr int EPL = 4, BYTES = 4; };
+template <> struct StateTraits<ST_BF16> { static constexpr int EPL = 8, BYTES = 2; };
+template <> struct StateTraits<ST_FP8> { static constexpr int EPL = 16, BYTES = 1; };
+
+// Streaming 16-byte load/store: the state is touched once per launch, so it
+// should not displace anything in L1/L2 ("evict first").
+__device__ __forceinline__ uint4 ld_stream16(const void* p) {
+  return __ldcs(reinterpret_cast<const uint4*>(p));
+}
+__device__ __forceinline__ void st_stream16(void* p, uint4 v) {
+  __stcs(reinterpret_cast<uint4*>(p), v);
+}
+
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+
+// Round to the nearest bf16 (ties to even) and keep it as fp32.
+__device__ __forceinline__ float round_bf16(float x) {
+  return __bfloat162float(__float2bfloat16_rn(x));
+}
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  uint32_t l = __bfloat16_as_ushort(__float2bfloat16_rn(lo));
+  uint32_t h = __bfloat16_as_ushort(__float2bfloat16_rn(hi));
+  return l | (h << 16);
+}
+
+// fp8 E4M3 pair <-> float2 (low byte = .x). Hardware conversions: decode is
+// exact (through half); encode rounds to nearest even and saturates to 448.
+__device__ __forceinline__ float2 e4m3x2_to_float2(uint16_t pair) {
+  const __half2 h(__nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(pair), __NV_E4M3));
+  return __half22float2(h);
+}
+__device__ __forceinline__ uint16_t float2_to_e4m3x2(float x, float y) {
+  return static_cast<uint16_t>(__nv_cvt_float2_to_fp8x2(make_float2(x, y), __NV_SATFINITE, __NV_E4M3));
+}
+
+// Decode 16 stored bytes into EPL floats (fp8 codes are returned unscaled).
+template <int SDT>
+__device__ __forceinline__ void decode16(uint4 raw, float* x) {
+  const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+  if constexpr (SDT == ST_F32) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) x[i] = __uint_as_float(w[i]);
+  } else if constexpr (SDT == ST_BF16) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) { x[2 * i] = bf16_lo(w[i]); x[2 * i + 1] = bf16_hi(w[i]); }
+  } else {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      float2 a = e4m3x2_to_float2(static_cast<uint16_t>(w[i] & 0xffffu));
+      float2 b = e4m3x2_to_float2(static_cast<uint16_t>(w[i] >> 16));
+      x[4 * i] = a.x; x[4 * i + 1] = a.y; x[4 * i + 2] = b.x; x[4 * i + 3] = b.y;
+    }
+  }
+}
+
+// Encode EPL floats into 16 stored bytes. For fp8 the caller passes x * r.
+template <int SDT>
+__device__ __forceinline__ uint4 encode16(const float* x) {
+  uint32_t w[4];
+  if constexpr (SDT == ST_F32) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) w[i] = __float_as_uint(x[i]);
+  } else if constexpr (SDT == ST_BF16) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) w[i] = pack_bf16x2(x[2 * i], x[2 * i + 1]);
+  } else {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      uint32_t lo = float2_to_e4m3x2(x[4 * i], x[4 * i + 1]);
+      uint32_t hi = float2_to_e4m3x2(x[4 * i + 2], x[4 * i + 3]);
+      w[i] = lo | (hi << 16);
+    }
+  }
+  return make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+// fp8 tile scale from the tile's amax: s = amax / 448 and r = 1 / s, both
+// correctly rounded; a zero tile (or one whose r overflows) stores s = 0 and
+// codes 0 (signalled by r = 0).
+__device__ __forceinline__ void fp8_scale_of(float amax, float& s, float& r) {
+  s = __fdiv_rn(amax, kE4M3Max);
+  r = __frcp_rn(s);
+  if (!(amax > 0.0f) || isinf(r)) { s = 0.0f; r = 0.0f; }
+}
+// The value handed to the E4M3 encoder: x * r, and +0 for a zero tile (so
+// that negative inputs do not encode as -0).
+__device__ __forceinline__ float fp8_prescale(float x, float r) {
+  return r == 0.0f ? 0.0f : __fmul_rn(x, r);
+}
+
+// ---------------------------------------------------------------------------
+// token inputs
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ float ld_in1(const void* base, int64_t i, bool bf16) {
+  return bf16 ? __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(base)[i])
+              : reinterpret_cast<const float*>(base)[i];
+}
+
+// N contiguous input elements starting at element i (i a multiple of N,
+// base 16-byte aligned), widened to fp32.
+template <int N>
+__device__ __forceinline__ void ld_in_vec(const void* base, int64_t i, bool bf16, float* x) {
+  if (bf16) {
+    const __nv_bfloat16* p = reinterpret_cast<const __nv_bfloat16*>(base) + i;
+    if constexpr (N % 8 == 0) {
+#pragma unroll
+      for (int c = 0; c < N / 8; ++c) {
+        uint4 r = reinterpret_cast<const uint4*>(p)[c];
+        const uint32_t w[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) { x[8 * c + 2 * j] = bf16_lo(w[j]); x[8 * c + 2 * j + 1] = bf16_hi(w[j]); }
+      }
+    } else if constexpr (N == 4) {
+      uint2 r = *reinterpret_cast<const uint2*>(p);
+      x[0] = bf16_lo(r.x); x[1] = bf16_hi(r.x); x[2] = bf16_lo(r.y); x[3] = bf16_hi(r.y);
+    } else if constexpr (N == 2) {
+      uint32_t r = *reinterpret_cast<const uint32_t*>(p);
+      x[0] = bf16_lo(r); x[1] = bf16_hi(r);
+    } else {
+#pragma unroll
+      for (int j = 0; j < N; ++j) x[j] = __bfloat162float(p[j]);
+    }
+  } else {
+    const float* p = reinterpret_cast<const float*>(base) + i;
+    if constexpr (N % 4 == 0) {
+#pragma unroll
+      for (int c = 0; c < N / 4; ++c) {
+        float4 r = reinterpret_cast<const float4*>(p)[c];
+        x[4 * c] = r.x; x[4 * c + 1] = r.y; x[4 * c + 2] = r.z; x[4 * c + 3] = r.w;
+      }
+    } else if constexpr (N == 2) {
+      float2 r = *reinterpret_cast<const float2*>(p);
+      x[0] = r.x; x[1] = r.y;
+    } else {
+#pragma unroll
+      for (int j = 0; j < N; ++j) x[j] = p[j];
+    }
+  }
+}
+
+__device__ __forceinline__ void st_out1(void* base, int64_t i, float x, bool bf16) {
+  if (bf16) reinterpret_cast<__nv_bfloat16*>(base)[i] = __float2bfloat16_rn(x);
+  else reinterpret_cast<float*>(base)[i] = x;
+}
+
+// ---------------------------------------------------------------------------
+// activations (fp32)
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ float softplus_f(float x) {
+  return fmaxf(x, 0.0f) + log1pf(expf(-fabsf(x)));
+}
+// alpha = exp(-exp(A_log) * softplus(x)), x = gate pre-activation + dt_bias
+__device__ __forceinline__ float decay_of(float exp_A_log, float x) {
+  return expf(-exp_A_log * softplus_f(x));
+}
+__device__ __forceinline__ float sigmoid_f(float x) { return 1.0f / (1.0f + expf(-x)); }
+
+template <int LANES>
+__device__ __forceinline__ float group_sum(float x) {
+#pragma unroll
+  for (int o = LANES / 2; o > 0; o >>= 1) x += __shfl_xor_sync(kFull, x, o);
+  return x;
+}
+template <int LANES>
+__device__ __forceinline__ float group_max(float x) {
+#pragma unroll
+  for (int o = LANES / 2; o > 0; o >>= 1) x = fmaxf(x, __shfl_xor_sync(kFull, x, o));
+  return x;
+}
+
+// ---------------------------------------------------------------------------
+// unit resolution
+// ---------------------------------------------------------------------------
+enum UnitStatus : int { U_OK = 0, U_PAD = 1, U_SKIP = 2 };
+
+struct Unit {
+  int64_t src, dst;  // pool slot (or page) read and written
+  int tok0, tok1;    // token range
+  int status;
+  int err;
+};
+
+__device__ __forceinline__ int64_t ld_index(const void* base, int64_t i, bool i64) {
+  return i64 ? reinterpret_cast<const int64_t*>(base)[i]
+             : static_cast<int64_t>(reinterpret_cast<const int32_t*>(base)[i]);
+}
+
+// Copy-on-new-page rule of a paged decode (flashinfer gdn_paged, description):
+// the decoded token sits in the sequence's last page; if it opens that page
+// (last_page_len == 1) the state is read from the page before it, otherwise
+// the last page is read and updated in place.
+__device__ __forceinline__ void resolve_page_rows(const void* indices, const void* indptr,
+                                                  const void* lastlen, bool i64, int64_t nnz,
+                                                  int64_t num_pages, int page_size, int b,
+                                                  int64_t& read, int64_t& write, int& err) {
+  read = write = -1;
+  const int64_t p0 = ld_index(indptr, b, i64);
+  const int64_t p1 = ld_index(indptr, b + 1, i64);
+  const int64_t len = ld_index(lastlen, b, i64);
+  if (p0 < 0 || p1 > nnz) { err |= E_PAGE_RANGE; return; }
+  if (p1 <= p0 || len < 1 || (page_size > 0 && len > page_size)) { err |= E_PAGE_TABLE; return; }
+  if (len == 1 && p1 - 1 <= p0) { err |= E_PAGE_TABLE; return; }
+  const int64_t w = ld_index(indices, p1 - 1, i64);
+  const int64_t r = (len == 1) ? ld_index(indices, p1 - 2, i64) : w;
+  if (w < 0 || w >= num_pages || r < 0 || r >= num_pages) { err |= E_PAGE_RANGE; return; }
+  read = r;
+  write = w;
+}
+
+template <int IDX>
+__device__ __forceinline__ Unit resolve_unit(const StepParams& p, int b) {
+  Unit u;
+  u.status = U_OK;
+  u.err = 0;
+  const bool i64 = (p.flags & F_IDX64) != 0;
+  if constexpr (IDX == IDX_SLOTS) {
+    if (p.flags & F_VARLEN) {
+      const int32_t* cu = reinterpret_cast<const int32_t*>(p.indptr);
+      u.tok0 = cu[b];
+      u.tok1 = cu[b + 1];
+      if (u.tok0 < 0 || u.tok1 < u.tok0 || u.tok1 > p.total_tokens) {
+        u.err |= E_SEQLENS;
+        u.status = U_SKIP;
+        return u;
+      }
+    } else {
+      u.tok0 = b * p.T;
+      u.tok1 = u.tok0 + p.T;
+    }
+    const int64_t s = ld_index(p.idx, b, i64);
+    u.src = u.dst = s;
+    if (s < 0) u.status = U_PAD;
+    else if (s >= p.num_slots) { u.status = U_PAD; u.err |= E_SLOT_RANGE; }
+  } else {
+    u.tok0 = b;
+    u.tok1 = b + 1;
+    if (p.rows != nullptr) {
+      u.src = p.rows[2 * b];
+      u.dst = p.rows[2 * b + 1];
+      if (u.src < 0 || u.dst < 0) u.status = U_PAD;
+      else if (u.src >= p.num_slots || u.dst >= p.num_slots) { u.status = U_PAD; u.err |= E_PAGE_RANGE; }
+    } else {
+      resolve_page_rows(p.idx, p.indptr, p.lastlen, i64, p.nnz, p.num_slots, p.page_size, b,
+                        u.src, u.dst, u.err);
+      if (u.err) u.status = U_PAD;
+    }
+  }
+  return u;
+}
+
+__device__ __forceinline__ void raise_err(int32_t* err, int bits) {
+  if (err != nullptr && bits != 0) atomicOr(err, bits);
+}
+
+}  // namespace gdn

@@ -1,0 +1,265 @@
+"""Shared drivers of the GPU parity tests: build one case from the seeded
+generators, run it through the C ABI (via the Python binding) and through the
+oracle on the same values, and compare.
+
+Tolerances (max relative error per (sequence, value head) slice,
+max|x - ref| / max|ref|): fp32 state 1e-4 on outputs and states; bf16 state
+2e-2; fp8 state: outputs 1e-4 (working readout reads the fp32 state), stored
+codes within one E4M3 step of the oracle's after dequantisation and >= 99.9%
+identical. bf16 outputs add the bf16 rounding of the output, 2^-8.
+"""
+
+from __future__ import annotations
+
+import math
+
+import numpy as np
+import torch
+
+import gated_delta_rule_80_b200 as G
+import workloads as W
+from oracle import formats
+from oracle import gdn as O
+
+TOL = {"f32": 1e-4, "bf16": 2e-2, "fp8_e4m3": 1e-4}
+BF16_OUT = 2.0 ** -8
+
+
+def dev(x: np.ndarray, dtype=None):
+    t = torch.from_numpy(np.ascontiguousarray(x))
+    if dtype is not None:
+        t = t.to(dtype)
+    return t.cuda()
+
+
+def dev_in(x: np.ndarray, in_dtype: str):
+    return dev(x.astype(np.float32), W.torch_dtype(in_dtype))
+
+
+def slice_rel_err(x: np.ndarray, ref: np.ndarray) -> float:
+    x = np.asarray(x, np.float64)
+    ref = np.asarray(ref, np.float64)
+    den = max(float(np.max(np.abs(ref))), 1e-30)
+    return float(np.max(np.abs(x - ref))) / den
+
+
+def host(t: torch.Tensor) -> np.ndarray:
+    if t.dtype == torch.bfloat16:
+        return t.float().cpu().numpy()
+    return t.cpu().numpy()
+
+
+def pool_host(pool: torch.Tensor) -> np.ndarray:
+    """Device pool -> numpy in the oracle's stored representation."""
+    if pool.dtype == torch.bfloat16:
+        return pool.view(torch.int16).cpu().numpy().view(np.uint16)
+    return pool.cpu().numpy()
+
+
+def check_outputs(out_gpu: np.ndarray, out_ref: np.ndarray, units, slicer, tol: float, out_dtype: str):
+    """units: iterable of (b, hv); slicer(arr, b, hv) -> the slice."""
+    worst = 0.0
+    lim = tol + (BF16_OUT if out_dtype == "bf16" else 0.0)
+    for (b, hv) in units:
+        ref = slicer(out_ref, b, hv)
+        if ref.size == 0:
+            continue
+        e = slice_rel_err(slicer(out_gpu, b, hv), ref)
+        worst = max(worst, e)
+        assert e <= lim, f"output slice (b={b}, hv={hv}): rel err {e:.3g} > {lim:.3g}"
+    return worst
+
+
+def check_state(pool_after: np.ndarray, scales_after, writes, state_dtype: str, layout: str, block_v=64):
+    """Compare every written (slot, hv) state with the oracle's."""
+    worst = 0.0
+    n_codes = n_same = 0
+    for (slot, hv), (st_ref, sc_ref) in writes.items():
+        got = pool_after[slot, hv]
+        if state_dtype == "f32":
+            e = slice_rel_err(got, st_ref)
+        elif state_dtype == "bf16":
+            e = slice_rel_err(formats.bf16_bits_to_f32(got), formats.bf16_bits_to_f32(st_ref))
+        else:
+            sc_got = scales_after[slot, hv]
+            assert np.allclose(sc_got, sc_ref, rtol=1e-5, atol=0), (slot, hv, sc_got, sc_ref)
+            kv_got = O._to_kv(got, layout)
+            kv_ref = O._to_kv(st_ref, layout)
+            deq_got = formats.dequantize_state(kv_got, sc_got, block_v).astype(np.float64)
+            deq_ref = formats.dequantize_state(kv_ref, sc_ref, block_v).astype(np.float64)
+            # one E4M3 step at the larger of the two magnitudes, in units of the tile scale
+            a = np.maximum(np.abs(deq_got), np.abs(deq_ref)) / np.repeat(np.maximum(sc_ref, 1e-38), block_v)[None, :]
+            step = np.exp2(np.maximum(np.floor(np.log2(np.maximum(a, 1e-30))), -6) - 3)
+            lim = step * np.repeat(sc_ref, block_v)[None, :] * 1.0001 + 1e-30
+            assert np.all(np.abs(deq_got - deq_ref) <= lim), f"fp8 state (slot={slot}, hv={hv}) off by > 1 step"
+            n_codes += got.size
+            n_same += int(np.sum(got == st_ref))
+            e = slice_rel_err(deq_got, deq_ref)
+            worst = max(worst, e)
+            continue
+        worst = max(worst, e)
+        assert e <= TOL[state_dtype], f"state (slot={slot}, hv={hv}): rel err {e:.3g}"
+    if n_codes:
+        assert n_same / n_codes >= 0.999, f"only {n_same / n_codes:.5f} of fp8 codes identical"
+    return worst
+
+
+def check_untouched(pool_before: np.ndarray, pool_after: np.ndarray, written_keys, scales_before=None,
+                    scales_after=None):
+    """Every (slot, hv) that is not written is bit-identical."""
+    mask = np.ones(pool_before.shape[:2], dtype=bool)
+    for (slot, hv) in written_keys:
+        mask[slot, hv] = False
+    a = pool_before[mask].view(np.uint8)
+    b = pool_after[mask].view(np.uint8)
+    assert np.array_equal(a, b), "a state that should be untouched changed"
+    if scales_before is not None:
+        assert np.array_equal(scales_before[mask].view(np.uint32), scales_after[mask].view(np.uint32))
+
+
+# ----------------------------------------------------------------------------
+# GDN slot pool case
+# ----------------------------------------------------------------------------
+
+def gdn_slots_case(seed, B, T, H, HV, K, V, num_slots, layout="V_FIRST", state_dtype="f32",
+                   in_dtype="bf16", out_dtype="f32", index_dtype="i32", readout="working",
+                   indices=None, use_qk_l2norm=True, scale=None, tokens=None, block_v=64,
+                   check=True, units=None):
+    """Run one GDN slot decode on the GPU and the oracle; assert parity. Returns a dict."""
+    t = tokens or W.gdn_tokens(seed, B, T, H, HV, K, V, in_dtype)
+    idx = np.asarray(indices if indices is not None else W.slot_indices(seed, B, num_slots), np.int64)
+    live = [int(s) for s in idx if 0 <= s < num_slots]
+    exact = set(live) if units is None else {int(idx[b]) for b, _ in units if 0 <= idx[b] < num_slots}
+    pool, scales = W.device_pool(seed, num_slots, HV, K, V, layout, state_dtype, block_v,
+                                 exact_slots=sorted(exact))
+    before = pool_host(pool)
+    sc_before = scales.cpu().numpy() if scales is not None else None
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out = G.gdn_decode_slots(
+        dev_in(t["q"], in_dtype), dev_in(t["k"], in_dtype), dev_in(t["v"], in_dtype),
+        dev_in(t["a"], in_dtype), dev_in(t["b"], in_dtype), dev(t["A_log"]), dev(t["dt_bias"]),
+        pool, dev(idx.astype(np.int32 if index_dtype == "i32" else np.int64)), state_scales=scales,
+        state_layout=layout, block_v=block_v, scale=scale, use_qk_l2norm=use_qk_l2norm,
+        output_dtype=W.torch_dtype(out_dtype), readout=readout, err_flags=err)
+    torch.cuda.synchronize()
+    after = pool_host(pool)
+    sc_after = scales.cpu().numpy() if scales is not None else None
+    res = dict(out=host(out), pool_before=before, pool_after=after, scales_before=sc_before,
+               scales_after=sc_after, err=int(err.item()), idx=idx, tokens=t)
+    if not check:
+        return res
+    ref_out, writes = O.gdn_decode_slots(
+        t["q"], t["k"], t["v"], t["a"], t["b"], t["A_log"], t["dt_bias"], before, idx,
+        layout=layout, state_dtype=state_dtype, state_scales=sc_before, block_v=block_v,
+        scale=scale, use_qk_l2norm=use_qk_l2norm, readout_mode=readout, num_slots=num_slots,
+        units=units)
+    todo = [(b, hv) for b in range(B) for hv in range(HV)] if units is None else units
+    res["out_err"] = check_outputs(res["out"], ref_out, todo, lambda x, b, hv: x[b, :, hv, :],
+                                   TOL[state_dtype], out_dtype)
+    res["state_err"] = check_state(after, sc_after, writes, state_dtype, layout, block_v)
+    written = {(s, hv) for s in live for hv in range(HV)} if T > 0 else set()
+    check_untouched(before, after, written, sc_before, sc_after)
+    res["writes"] = writes
+    res["ref_out"] = ref_out
+    return res
+
+
+# ----------------------------------------------------------------------------
+# GDN paged case
+# ----------------------------------------------------------------------------
+
+def gdn_paged_case(seed, B, H, HV, K, V, page_size, max_len, n_share, share_pages, force_lens=None,
+                   state_dtype="f32", in_dtype="bf16", out_dtype="f32", index_dtype="i32",
+                   use_slots=False, units=None, spare_pages=0, readout="working", layout="V_FIRST"):
+    pt = W.paged_table(seed, B, page_size, max_len, n_share, share_pages, force_lens,
+                       spare_pages).cast(index_dtype)
+    t = W.gdn_tokens(seed, B, 1, H, HV, K, V, in_dtype)
+    rows = O.paged_decode_slots(pt.page_indices, pt.page_indptr, pt.last_page_len)
+    touched = sorted(set(rows.reshape(-1).tolist()))
+    pool, scales = W.device_pool(seed, pt.num_pages, HV, K, V, layout, state_dtype,
+                                 exact_slots=touched)
+    snap = pool.clone()
+    sc_snap = scales.clone() if scales is not None else None
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    pi, pp, pl = dev(pt.page_indices), dev(pt.page_indptr), dev(pt.last_page_len)
+    slots = None
+    if use_slots:
+        slots = G.gdn_paged_decode_slots(pi, pp, pl, pt.num_pages, page_size, err_flags=err)
+    out = G.gdn_decode_paged(
+        dev_in(t["q"], in_dtype), dev_in(t["k"], in_dtype), dev_in(t["v"], in_dtype),
+        dev(t["A_log"]), dev_in(t["a"], in_dtype), dev(t["dt_bias"]), dev_in(t["b"], in_dtype),
+        state_pool=pool, page_indices=pi, page_indptr=pp, last_page_len=pl, slots=slots,
+        state_scales=scales, state_layout=layout, page_size=page_size,
+        output_dtype=W.torch_dtype(out_dtype), readout=readout, err_flags=err)
+    torch.cuda.synchronize()
+    res = dict(err=int(err.item()), table=pt, rows=rows)
+    if slots is not None:
+        res["slots"] = slots.cpu().numpy()
+    # the oracle reads only the pages it needs, from the generator
+    states, sc = W.host_pool(seed, touched, HV, K, V, layout, state_dtype)
+    all_units = [(b, hv) for b in range(B) for hv in range(HV)]
+    todo = all_units if units is None else units
+    ref_out, writes = O.gdn_decode_paged(
+        t["q"], t["k"], t["v"], t["a"], t["b"], t["A_log"], t["dt_bias"], states, pt.page_indices,
+        pt.page_indptr, pt.last_page_len, state_dtype=state_dtype, state_scales=sc,
+        readout_mode=readout, units=todo)
+    out_h = host(out)
+    res["out_err"] = check_outputs(out_h, ref_out, todo, lambda x, b, hv: x[b, 0, hv, :],
+                                   TOL[state_dtype], out_dtype)
+    # written pages: compare the sampled units; every other page must be bit-identical
+    write_pages = sorted(set(rows[:, 1].tolist()))
+    wp = torch.tensor(write_pages, device="cuda")
+    after_w = pool_host(pool[wp])
+    sc_after_w = scales[wp].cpu().numpy() if scales is not None else None
+    pos = {p: i for i, p in enumerate(write_pages)}
+    sub_writes = {(pos[p], hv): w for (p, hv), w in writes.items()}
+    res["state_err"] = check_state(after_w, sc_after_w, sub_writes, state_dtype, layout)
+    keep = torch.ones(pt.num_pages, dtype=torch.bool, device="cuda")
+    keep[wp] = False
+    assert torch.equal(pool[keep], snap[keep]), "a page that is not a write page changed"
+    if scales is not None:
+        assert torch.equal(scales[keep], sc_snap[keep])
+    res["write_pages"] = write_pages
+    return res
+
+
+# ----------------------------------------------------------------------------
+# KDA varlen case
+# ----------------------------------------------------------------------------
+
+def kda_case(seed, B, Hk, HV, K, V, num_slots, max_len, layout="K_FIRST", state_dtype="f32",
+             in_dtype="bf16", out_dtype="f32", beta_mode="logits", cu=None, indices=None,
+             readout="working", tokens=None):
+    cu = np.asarray(cu if cu is not None else W.varlen_offsets(seed, B, max_len), np.int32)
+    total = int(cu[-1])
+    t = tokens or W.kda_tokens(seed, total, Hk, HV, K, V, in_dtype)
+    if beta_mode == "probability":
+        t = dict(t, beta_logits=W.as_dtype_values(1.0 / (1.0 + np.exp(-t["beta_logits"])), in_dtype))
+    idx = np.asarray(indices if indices is not None else W.slot_indices(seed, B, num_slots), np.int64)
+    live = sorted(set(int(s) for s in idx if 0 <= s < num_slots))
+    pool, scales = W.device_pool(seed, num_slots, HV, K, V, layout, state_dtype, exact_slots=live)
+    before = pool_host(pool)
+    sc_before = scales.cpu().numpy() if scales is not None else None
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out = G.kda_decode_varlen(
+        dev_in(t["q"], in_dtype), dev_in(t["k"], in_dtype), dev_in(t["v"], in_dtype),
+        dev_in(t["raw_gate"], in_dtype), dev_in(t["beta_logits"], in_dtype), dev(t["a_log"]),
+        dev(t["dt_bias"]), dev(cu), pool, dev(idx.astype(np.int32)),
+        output_dtype=W.torch_dtype(out_dtype), beta_mode=beta_mode, state_layout=layout,
+        state_scales=scales, readout=readout, err_flags=err)
+    torch.cuda.synchronize()
+    after = pool_host(pool)
+    sc_after = scales.cpu().numpy() if scales is not None else None
+    ref_out, writes = O.kda_decode_varlen(
+        t["q"], t["k"], t["v"], t["raw_gate"], t["beta_logits"], t["a_log"], t["dt_bias"], cu, before, idx,
+        layout=layout, state_dtype=state_dtype, state_scales=sc_before, beta_mode=beta_mode,
+        readout_mode=readout, num_slots=num_slots)
+    out_h = host(out)
+    units = [(b, hv) for b in range(B) for hv in range(HV)]
+    res = dict(out=out_h, err=int(err.item()), writes=writes, pool_before=before, pool_after=after, cu=cu)
+    res["out_err"] = check_outputs(out_h, ref_out, units,
+                                   lambda x, b, hv: x[int(cu[b]):int(cu[b + 1]), hv, :],
+                                   TOL[state_dtype], out_dtype)
+    res["state_err"] = check_state(after, sc_after, writes, state_dtype, layout)
+    check_untouched(before, after, writes.keys(), sc_before, sc_after)
+    return res
