@@ -1,0 +1,518 @@
+"""Benchmark of gated delta-rule decode on B200.
+
+Default workload: slot-pool GDN decode, T=1, B=64 sequences, H=16 key heads,
+HV=32 value heads, K=V=128, bf16 q/k/v/a/b, fp32 state pool
+[256, 32, 128, 128] (V_FIRST), bf16 output. One step = one decode call over
+the batch: every sequence's state is read, advanced one token and written
+back in place. Steps rotate over 4 disjoint sets of 64 slots (512 MiB of
+state per cycle, 4x the L2), so no step finds its state in L2.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl b200|reference]
+                    [--workload slots|paged|kda|fp8|tiny]
+
+Prints one JSON line (rank 0). Under torchrun each rank runs its own batch
+on its own GPU (weak scaling; the sequences are independent, no data-path
+collective); timing is the max over ranks.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import re
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+import workloads as W  # noqa: E402
+
+METRIC = "decode tokens/s and achieved HBM GB/s (% of ~8 TB/s) at 1×B200, by config"
+L2_BYTES = 126 * 2 ** 20
+PROFILES = os.path.join(ROOT, "profiles")
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["b200", "reference"], default="b200")
+    ap.add_argument("--workload", choices=["slots", "paged", "kda", "fp8", "tiny"], default="slots")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    return ap.parse_args()
+
+
+# ----------------------------------------------------------------------------
+# distributed plumbing
+# ----------------------------------------------------------------------------
+
+def dist_setup(gpus):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ----------------------------------------------------------------------------
+# clocks during the timed region (NVML)
+# ----------------------------------------------------------------------------
+
+class ClockSampler:
+    REASONS = {"hw_slowdown": 0x8, "hw_thermal_slowdown": 0x40, "sw_thermal_slowdown": 0x20,
+               "sw_power_cap": 0x4, "hw_power_brake_slowdown": 0x80}
+
+    def __init__(self, index):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self._stop = threading.Event()
+        self._on = threading.Event()
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            try:   # match the CUDA device to its NVML handle by UUID
+                uuid = "GPU-" + str(torch.cuda.get_device_properties(index).uuid)
+                self.h = pynvml.nvmlDeviceGetHandleByUUID(uuid)
+            except Exception:
+                self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self.nv = None
+
+    def _run(self):
+        while not self._stop.is_set():
+            if self._on.is_set():
+                try:
+                    self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+                    r = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                    for name, bit in self.REASONS.items():
+                        if r & bit:
+                            self.reasons.add(name)
+                except Exception:
+                    pass
+            time.sleep(0.005)
+
+    def __enter__(self):
+        if self.nv is not None:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def timing(self, on: bool):
+        (self._on.set if on else self._on.clear)()
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self.nv is not None:
+            self.t.join()
+
+    def summary(self):
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "samples": len(self.samples),
+                "reasons": sorted(self.reasons)}
+
+
+# ----------------------------------------------------------------------------
+# workloads on the device
+# ----------------------------------------------------------------------------
+
+def in_t(x, dt):
+    return torch.from_numpy(np.ascontiguousarray(x)).to(W.torch_dtype(dt)).cuda()
+
+
+def describe_slots(w: W.Workload) -> str:
+    return (f"slot-pool GDN decode T={w.T}: B={w.B}, H={w.H}, HV={w.HV}, K=V={w.K}, {w.in_dtype} q/k/v/a/b, "
+            f"{w.state_dtype} state_pool [{w.num_slots},{w.HV},{w.V},{w.K}] {w.layout}, bf16 output")
+
+
+class SlotsRun:
+    """GDN slot pool, T=1 (the 'slots' and 'fp8' workloads)."""
+
+    def __init__(self, w: W.Workload, rank: int):
+        import gated_delta_rule_80_b200 as G
+        self.G, self.w = G, w
+        seed = w.seed + 1000 * rank
+        self.seed = seed
+        t = W.gdn_tokens(seed, w.B, w.T, w.H, w.HV, w.K, w.V, w.in_dtype)
+        self.host_tokens = t
+        self.q, self.k, self.v = in_t(t["q"], w.in_dtype), in_t(t["k"], w.in_dtype), in_t(t["v"], w.in_dtype)
+        self.a, self.b = in_t(t["a"], w.in_dtype), in_t(t["b"], w.in_dtype)
+        self.A_log, self.dt_bias = in_t(t["A_log"], "f32"), in_t(t["dt_bias"], "f32")
+        self.pool, self.scales = W.device_pool(seed, w.num_slots, w.HV, w.K, w.V, w.layout, w.state_dtype,
+                                               w.block_v)
+        self.n_rot = w.num_slots // w.B
+        self.idx = [torch.from_numpy(W.slot_indices(seed, w.B, w.num_slots, r).astype(np.int32)).cuda()
+                    for r in range(self.n_rot)]
+        self.out = torch.empty((w.B, w.T, w.HV, w.V), dtype=torch.bfloat16, device="cuda")
+        sb = {"f32": 4, "bf16": 2, "fp8_e4m3": 1}[w.state_dtype]
+        state = 2 * w.HV * w.K * w.V * sb + (2 * w.HV * (w.V // w.block_v) * 4 if w.state_dtype == "fp8_e4m3" else 0)
+        ib = 2 if w.in_dtype == "bf16" else 4
+        io = (2 * w.H * w.K + w.HV * w.V + 2 * w.HV) * ib + w.HV * w.V * 2 + 4
+        self.tokens_per_step = w.B * w.T
+        # the state is read and written once per call, token inputs/outputs once per token
+        self.bytes_per_step = state * w.B + io * w.B * w.T + w.HV * 8   # + A_log, dt_bias
+        self.bytes_per_token = self.bytes_per_step / self.tokens_per_step
+        self.l2_note = (f"rotating {self.n_rot} disjoint slot sets "
+                        f"({self.n_rot * w.B * 2 * w.HV * w.K * w.V * sb // 2 // 2**20} MiB of state per cycle)"
+                        if self.n_rot > 1 else "state touched per step > L2 (every slot every step)")
+
+    def step(self, i):
+        self.G.gdn_decode_slots(self.q, self.k, self.v, self.a, self.b, self.A_log, self.dt_bias, self.pool,
+                                self.idx[i % self.n_rot], state_scales=self.scales, state_layout=self.w.layout,
+                                block_v=self.w.block_v, output=self.out)
+
+    def e2e_setup(self):
+        pin = lambda x: x.cpu().pin_memory()
+        self.h_in = [pin(x) for x in (self.q, self.k, self.v, self.a, self.b)]
+        self.h_idx = [pin(x) for x in self.idx]
+        self.d_in = [torch.empty_like(x) for x in (self.q, self.k, self.v, self.a, self.b)]
+        self.d_idx = torch.empty_like(self.idx[0])
+        self.h_out = torch.empty(self.out.shape, dtype=self.out.dtype).pin_memory()
+        self.h2d = sum(x.numel() * x.element_size() for x in self.h_in) + self.h_idx[0].numel() * 4
+        self.d2h = self.h_out.numel() * self.h_out.element_size()
+
+    def e2e_step(self, i):
+        for d, h in zip(self.d_in, self.h_in):
+            d.copy_(h, non_blocking=True)
+        self.d_idx.copy_(self.h_idx[i % self.n_rot], non_blocking=True)
+        q, k, v, a, b = self.d_in
+        self.G.gdn_decode_slots(q, k, v, a, b, self.A_log, self.dt_bias, self.pool, self.d_idx,
+                                state_scales=self.scales, state_layout=self.w.layout, block_v=self.w.block_v,
+                                output=self.out)
+        self.h_out.copy_(self.out, non_blocking=True)
+
+    def describe(self):
+        return describe_slots(self.w)
+
+    def cpu_baseline(self, seconds):
+        """The oracle on rank 0's first sequences, as many as fit the time budget."""
+        from threadpoolctl import threadpool_limits
+        from oracle import gdn as O
+        w, t = self.w, self.host_tokens
+        nb = min(w.B, 8)
+        idx = W.slot_indices(self.seed, w.B, w.num_slots, 0)[:nb]
+        states, scales = W.host_pool(self.seed, idx.tolist(), w.HV, w.K, w.V, w.layout, w.state_dtype, w.block_v)
+        sl = lambda x: x[:nb]
+        done, t0 = 0, time.perf_counter()
+        with threadpool_limits(limits=1):
+            while True:
+                O.gdn_decode_slots(sl(t["q"]), sl(t["k"]), sl(t["v"]), sl(t["a"]), sl(t["b"]), t["A_log"],
+                                   t["dt_bias"], states, idx, layout=w.layout, state_dtype=w.state_dtype,
+                                   state_scales=scales, block_v=w.block_v)
+                done += nb * w.T
+                el = time.perf_counter() - t0
+                if el >= seconds:
+                    break
+        return done / el, f"oracle gdn_decode_slots on {nb} of {w.B} sequences x {w.HV} heads, repeated " \
+                          f"{done // (nb * w.T)} times in {el:.1f} s"
+
+
+class PagedRun:
+    """GDN paged pool, one token (the 'paged' workload). Between timed steps
+    a read of a 512 MiB buffer evicts the pages from L2."""
+
+    def __init__(self, w: W.Workload, rank: int):
+        import gated_delta_rule_80_b200 as G
+        self.G, self.w = G, w
+        seed = w.seed + 1000 * rank
+        self.seed = seed
+        pt = W.paged_table(seed, w.B, w.page_size, w.max_len, w.n_share, w.share_pages).cast("i32")
+        self.pt = pt
+        t = W.gdn_tokens(seed, w.B, 1, w.H, w.HV, w.K, w.V, w.in_dtype)
+        self.host_tokens = t
+        self.q, self.k, self.v = in_t(t["q"], w.in_dtype), in_t(t["k"], w.in_dtype), in_t(t["v"], w.in_dtype)
+        self.a, self.b = in_t(t["a"], w.in_dtype), in_t(t["b"], w.in_dtype)
+        self.A_log, self.dt_bias = in_t(t["A_log"], "f32"), in_t(t["dt_bias"], "f32")
+        self.pool, self.scales = W.device_pool(seed, pt.num_pages, w.HV, w.K, w.V, w.layout, w.state_dtype)
+        self.pi = torch.from_numpy(pt.page_indices).cuda()
+        self.pp = torch.from_numpy(pt.page_indptr).cuda()
+        self.pl = torch.from_numpy(pt.last_page_len).cuda()
+        self.out = torch.empty((w.B, 1, w.HV, w.V), dtype=torch.bfloat16, device="cuda")
+        self.flush_buf = torch.empty(4 * L2_BYTES // 4, dtype=torch.float32, device="cuda")
+        ib = 2
+        self.bytes_per_token = 2 * w.HV * w.K * w.V * 4 + (2 * w.H * w.K + w.HV * w.V + 2 * w.HV) * ib \
+            + w.HV * w.V * 2 + 12
+        self.tokens_per_step = w.B
+        self.bytes_per_step = self.bytes_per_token * w.B + w.HV * 8
+        self.l2_note = "L2 evicted between timed steps by reading a 504 MiB buffer (untimed)"
+        self.needs_flush = True
+
+    def flush(self):
+        self.flush_buf.sum()
+
+    def step(self, i):
+        self.G.gdn_decode_paged(self.q, self.k, self.v, self.A_log, self.a, self.dt_bias, self.b,
+                                state_pool=self.pool, page_indices=self.pi, page_indptr=self.pp,
+                                last_page_len=self.pl, page_size=self.w.page_size, output=self.out)
+
+    def describe(self):
+        w = self.w
+        return (f"paged GDN decode T=1: B={w.B}, page_size={w.page_size}, lengths U[2,{w.max_len}], "
+                f"{w.n_share} sequences sharing {w.share_pages} full pages, HV={w.HV}, H={w.H}, K=V={w.K}, "
+                f"fp32 state_pool [{self.pt.num_pages},{w.HV},{w.V},{w.K}], int32 CSR, bf16 in/out")
+
+
+class KdaRun:
+    """KDA varlen (the 'kda' workload), 8 pool replicas rotated."""
+
+    def __init__(self, w: W.Workload, rank: int, layout=None):
+        import gated_delta_rule_80_b200 as G
+        self.G, self.w = G, w
+        seed = w.seed + 1000 * rank
+        self.layout = layout or w.layout
+        self.cu = W.varlen_offsets(seed, w.B, w.max_len)
+        total = int(self.cu[-1])
+        t = W.kda_tokens(seed, total, w.H, w.HV, w.K, w.V, w.in_dtype)
+        self.ins = [in_t(t[n], w.in_dtype) for n in ("q", "k", "v", "raw_gate", "beta_logits")]
+        self.a_log, self.dt_bias = in_t(t["a_log"], "f32"), in_t(t["dt_bias"], "f32")
+        self.cu_d = torch.from_numpy(self.cu).cuda()
+        self.idx = torch.from_numpy(W.slot_indices(seed, w.B, w.num_slots).astype(np.int32)).cuda()
+        self.n_rep = 8
+        self.pools = [W.device_pool(seed + r, w.num_slots, w.HV, w.K, w.V, self.layout, "f32")[0]
+                      for r in range(self.n_rep)]
+        self.out = torch.empty((total, w.HV, w.V), dtype=torch.bfloat16, device="cuda")
+        self.tokens_per_step = total
+        self.bytes_per_step = w.B * 2 * w.HV * w.K * w.V * 4 + total * (
+            (2 * w.H * w.K + w.HV * w.V + w.HV * w.K + w.HV) * 2 + w.HV * w.V * 2) + w.HV * (w.K + 1) * 4
+        self.bytes_per_token = self.bytes_per_step / total
+        self.l2_note = f"rotating {self.n_rep} pool replicas ({self.n_rep * w.num_slots * 2} MiB of state)"
+
+    def step(self, i):
+        q, k, v, g, bl = self.ins
+        self.G.kda_decode_varlen(q, k, v, g, bl, self.a_log, self.dt_bias, self.cu_d, self.pools[i % self.n_rep],
+                                 self.idx, state_layout=self.layout, output=self.out)
+
+    def describe(self):
+        w = self.w
+        return (f"KDA varlen decode: {w.B} sequences x U[1,{w.max_len}] tokens ({self.tokens_per_step} tokens), "
+                f"Hk=HV={w.HV}, K=V={w.K}, bf16 inputs, fp32 state_pool [{w.num_slots},{w.HV},{w.K},{w.V}] "
+                f"{self.layout}")
+
+
+def make_run(name, rank):
+    w = W.WORKLOADS[name]
+    if name in ("slots", "fp8", "tiny"):
+        return SlotsRun(w, rank)
+    if name == "paged":
+        return PagedRun(w, rank)
+    return KdaRun(w, rank)
+
+
+# ----------------------------------------------------------------------------
+# roofline bookkeeping
+# ----------------------------------------------------------------------------
+
+def source_digest():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "gated_delta_rule_80_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        if f.endswith((".cu", ".cuh")):
+            h.update(open(os.path.join(csrc, f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(workload):
+    """DRAM bytes per launch from the committed ncu summary of this workload,
+    or None when the kernel sources changed since it was taken."""
+    path = os.path.join(PROFILES, f"gdn_decode_{workload}_ncu.md")
+    if not os.path.exists(path):
+        return None
+    text = open(path).read()
+    dig = re.search(r"source_digest:\s*([0-9a-f]+)", text)
+    tb = re.search(r"dram_bytes_per_launch:\s*([0-9.e+]+)", text)
+    if not dig or not tb or dig.group(1) != source_digest():
+        return None
+    return float(tb.group(1))
+
+
+def measured_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        return float(json.load(open(path))["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+# ----------------------------------------------------------------------------
+# arms
+# ----------------------------------------------------------------------------
+
+def run_b200(args, world, rank, local):
+    import gated_delta_rule_80_b200 as G
+    G.lib()
+    run = make_run(args.workload, rank)
+    stream = torch.cuda.current_stream()
+    flush = getattr(run, "needs_flush", False)
+    # bring the clocks up before the measured warm-up
+    t_end = time.perf_counter() + 0.5
+    i = 0
+    while time.perf_counter() < t_end:
+        for _ in range(50):
+            run.step(i)
+            i += 1
+        torch.cuda.synchronize()
+    for j in range(args.warmup):
+        run.step(j)
+    torch.cuda.synchronize()
+    K = args.steps
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    with ClockSampler(local) as clk:
+        barrier(world)
+        torch.cuda.synchronize()
+        clk.timing(True)
+        for j in range(K):
+            if flush:
+                run.flush()
+            starts[j].record(stream)
+            run.step(j)
+            ends[j].record(stream)
+        torch.cuda.synchronize()
+        clk.timing(False)
+        barrier(world)
+    kern_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    if flush:
+        total_ms = sum(kern_ms)
+    else:
+        total_ms = starts[0].elapsed_time(ends[-1])
+    total_ms = max_over_ranks(total_ms, world)
+    ms_per_step = total_ms / K
+    kern_avg_ms = statistics.fmean(kern_ms)
+    value = world * run.tokens_per_step * K / (total_ms / 1e3)
+    peak, peak_kind = measured_peak()
+    achieved = run.bytes_per_step / (kern_avg_ms / 1e3) / 1e9
+    traffic = profiled_traffic(args.workload)
+
+    e2e = None
+    if not args.no_e2e and hasattr(run, "e2e_setup"):
+        run.e2e_setup()
+        for j in range(max(3, args.warmup)):
+            run.e2e_step(j)
+        torch.cuda.synchronize()
+        Ke = max(1, min(K, 500))
+        barrier(world)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for j in range(Ke):
+            run.e2e_step(j)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+        e_ms = max_over_ranks(e0.elapsed_time(e1), world)
+        e2e = {"value": world * run.tokens_per_step * Ke / (e_ms / 1e3), "unit": "tokens/s",
+               "h2d_bytes_per_step": run.h2d, "d2h_bytes_per_step": run.d2h, "steps": Ke}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and hasattr(run, "cpu_baseline"):
+        v, sample = run.cpu_baseline(args.cpu_seconds)
+        cpu = {"value": v, "unit": "tokens/s", "cores": 1, "kind": "oracle", "sample": sample}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f32", "data": "synthetic (seeded; no dataset on the pages)",
+            "config": {"workload": run.describe(), "tokens_per_step_per_gpu": run.tokens_per_step,
+                       "l2": run.l2_note, "parallelism": f"independent sequences per GPU x{world}"},
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                         "frac": achieved / peak, "traffic": traffic, "peak_kind": peak_kind,
+                         "algorithmic_bytes_per_launch": run.bytes_per_step,
+                         "kernel_avg_us": kern_avg_ms * 1e3, "frac_of_8TBps": achieved / 8000.0},
+            "clocks": clk.summary(),
+            "e2e": e2e,
+            "gpu_launches": K,
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+
+
+def run_reference(args, world, rank):
+    """The oracle as the reference arm (rank 0 only), each step a bounded
+    sample of the same workload."""
+    if rank != 0:
+        return
+    from threadpoolctl import threadpool_limits
+    from oracle import gdn as O
+    w = W.WORKLOADS["slots"]
+    nb = 4
+    t = W.gdn_tokens(w.seed, w.B, w.T, w.H, w.HV, w.K, w.V, w.in_dtype)
+    idx = W.slot_indices(w.seed, w.B, w.num_slots, 0)[:nb]
+    states, _ = W.host_pool(w.seed, idx.tolist(), w.HV, w.K, w.V, w.layout, w.state_dtype)
+    sl = lambda x: x[:nb]
+
+    def step():
+        O.gdn_decode_slots(sl(t["q"]), sl(t["k"]), sl(t["v"]), sl(t["a"]), sl(t["b"]), t["A_log"], t["dt_bias"],
+                           states, idx, layout=w.layout, state_dtype=w.state_dtype)
+
+    with threadpool_limits(limits=1):
+        for _ in range(args.warmup):
+            step()
+        K = min(args.steps, 200)
+        t0 = time.perf_counter()
+        for _ in range(K):
+            step()
+        el = time.perf_counter() - t0
+    value = nb * K / el
+    sample = f"oracle gdn_decode_slots on {nb} of {w.B} sequences x {w.HV} heads per step"
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+            "steps": K, "warmup": args.warmup, "ms_per_step": el / K * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": describe_slots(w)},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        rank = int(os.environ.get("RANK", "0"))
+        run_reference(args, int(os.environ.get("WORLD_SIZE", "1")), rank)
+        return
+    world, rank, local = dist_setup(args.gpus)
+    try:
+        run_b200(args, world, rank, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

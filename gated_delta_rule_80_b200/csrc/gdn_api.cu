@@ -5,6 +5,7 @@
 // the device nor the stream. The device is taken from the state pool's
 // pointer: this library links its own CUDA runtime, whose current device is
 // independent of the caller's.
+#include <algorithm>
 #include <climits>
 #include <cmath>
 #include <cstdint>
@@ -12,7 +13,7 @@
 #include <utility>
 
 #include "../../include/gdn.h"
-#include "gdn_step.cuh"
+#include "gdn_tile1.cuh"
 
 using namespace gdn;
 
@@ -74,8 +75,22 @@ int launch_status() {
   return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
 
+// Single-token GDN decode on a V_FIRST pool: one small CTA per tile.
+template <int SDT, int K, int IDX>
+int launch_tile1(StepParams p, int B, cudaStream_t s) {
+  using TS = Tile1Shape<SDT, K>;
+  p.n_vtiles = p.V / TS::VT;
+  const int64_t units = static_cast<int64_t>(B) * p.HV * p.n_vtiles;
+  if (units > INT_MAX) return GDN_ERR_INVALID_ARG;
+  step_tile1<SDT, K, IDX><<<static_cast<unsigned>(units), TS::NW * 32, 0, s>>>(p);
+  return launch_status();
+}
+
 template <int L, int SDT, int K, int GATE, int IDX>
 int launch_one(StepParams p, int B, cudaStream_t s) {
+  if constexpr (L == L_VFIRST && GATE == GATE_SCALAR) {
+    if (p.T == 1) return launch_tile1<SDT, K, IDX>(p, B, s);
+  }
   constexpr int VT = TileShape<SDT>::VT;
   constexpr int NT = TileShape<SDT>::NW * 32;
   p.n_vtiles = p.V / VT;

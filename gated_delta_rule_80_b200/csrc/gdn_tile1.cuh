@@ -1,0 +1,257 @@
+// Single-token GDN decode on V_FIRST pools: one short-lived CTA per
+// (sequence, value head, V-tile), kept small in registers so that many CTAs
+// per SM keep their state loads in flight.
+//
+// The state tile is VT rows of K contiguous elements (one value column of S
+// per row), a contiguous block in the pool. A CTA of NW warps issues every
+// 16-byte load of its tile at once, right after the (dependent) slot or page
+// resolution; the token prologue is computed while the loads are in flight.
+//
+// Per row (value column v) the step needs a_k = k.S[:, v] and a_q = q.S[:, v]
+// summed over the LPR lanes that hold the row. The 2 * NR partial sums of a
+// thread go through a reduce-scatter (halving exchanges, then a plain
+// butterfly), so each lane ends with one finished sum; k.S and q.S of a row
+// meet with one more exchange, the lane computes u and o for that row, and u
+// is broadcast back to the lanes that update the row. q and k are used raw
+// in the dot products and their norms are applied to the reduced sums:
+//     a_k = |k|^-1 (k.S),   a_q = scale |q|^-1 (q.S),   q^.k^ likewise,
+// then (single pass, S read once, written once)
+//     u = beta (v - alpha a_k),   o = alpha a_q + (q^.k^) u,
+//     S' = alpha S + k^ u^T.
+#pragma once
+
+#include "gdn_step.cuh"
+
+namespace gdn {
+
+template <int SDT, int K>
+struct Tile1Shape {
+  static constexpr int VT = (SDT == ST_FP8) ? 64 : 32;   // fp8: the [K, 64] scale tile
+  static constexpr int NW = (SDT == ST_FP8 && K > 32) ? 8 : 4;
+};
+
+// Reduce-scatter of N values over the lanes of a row group: each halving
+// stage (offset O) sends half of the kept values to the partner lane and
+// keeps the other half, the upper half where (li & O) != 0; once one value is
+// left the remaining stages are a plain butterfly. A lane ends with the full
+// group sum of value number li / (LPR / N0).
+template <int N, int O>
+struct ReduceScatter {
+  __device__ __forceinline__ static float run(float* x, int li) {
+    if constexpr (N > 1) {
+      const bool hi = (li & O) != 0;
+#pragma unroll
+      for (int i = 0; i < N / 2; ++i) {
+        const float keep = hi ? x[N / 2 + i] : x[i];
+        const float send = hi ? x[i] : x[N / 2 + i];
+        x[i] = keep + __shfl_xor_sync(kFull, send, O);
+      }
+      return ReduceScatter<N / 2, O / 2>::run(x, li);
+    } else {
+      float v = x[0];
+#pragma unroll
+      for (int o = O; o >= 1; o >>= 1) v += __shfl_xor_sync(kFull, v, o);
+      return v;
+    }
+  }
+};
+
+template <int SDT, int K, int IDX>
+__global__ void __launch_bounds__(Tile1Shape<SDT, K>::NW * 32)
+step_tile1(const StepParams p) {
+  using ST = StateTraits<SDT>;
+  constexpr int EPL = ST::EPL;
+  constexpr int LPR = K / EPL;  // lanes per stored row
+  static_assert(K % EPL == 0 && LPR >= 2 && LPR <= 32 && 32 % LPR == 0, "row must fit a warp");
+  constexpr int RPW = 32 / LPR;  // rows per warp instruction
+  constexpr int VT = Tile1Shape<SDT, K>::VT;
+  constexpr int NW = Tile1Shape<SDT, K>::NW;
+  constexpr int NR = VT / (NW * RPW);  // rows per thread
+  static_assert(NR >= 1 && NR * NW * RPW == VT, "tile must split evenly");
+  constexpr int NV = 2 * NR;           // k.S and q.S partial sums per thread
+  static_assert(NV <= LPR, "one finished sum per lane");
+  constexpr int REP = LPR / NV;        // lanes that end with the same sum
+
+  __shared__ float s_amax[NW];
+
+  const int lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5;
+  const int li = lane % LPR;
+  const int ri = lane / LPR;
+  const int vidx = li / REP;           // the sum this lane finishes
+  const int myrow = vidx >> 1;         // ... belongs to this of the thread's rows
+  const bool holds_q = (vidx & 1) != 0;
+  const int grp = lane - li;
+  const bool writer = !holds_q && (li % REP) == 0;
+  int unit = blockIdx.x;
+  const int tile = unit % p.n_vtiles;
+  unit /= p.n_vtiles;
+  const int hv = unit % p.HV;
+  const int b = unit / p.HV;           // T == 1: the token of sequence b is b
+  const int h = hv / (p.HV / p.H);
+  const int kofs = li * EPL;
+  const bool in_bf16 = (p.flags & F_IN_BF16) != 0;
+  const int row0 = tile * VT + warp * NR * RPW + ri;   // row jj is row0 + jj * RPW
+  const int myrow_v = row0 + myrow * RPW;
+
+  const Unit u = resolve_unit<IDX>(p, b);
+  if (threadIdx.x == 0) raise_err(p.err, u.err);
+  if (u.status == U_SKIP) return;
+  const int64_t out_at = ((int64_t)b * p.HV + hv) * p.V + myrow_v;
+  if (u.status == U_PAD) {
+    if (writer) st_out1(p.out, out_at, 0.0f, (p.flags & F_OUT_BF16) != 0);
+    return;
+  }
+
+  // all state loads first
+  const int64_t head_elems = (int64_t)K * p.V;
+  const char* src = reinterpret_cast<const char*>(p.pool) +
+                    ((u.src * p.HV + hv) * head_elems + (int64_t)row0 * K + kofs) * ST::BYTES;
+  uint4 raw[NR];
+#pragma unroll
+  for (int jj = 0; jj < NR; ++jj) raw[jj] = ld_stream16(src + (int64_t)jj * RPW * K * ST::BYTES);
+  [[maybe_unused]] float sc_in = 1.0f;
+  const int n_scale = p.V / VT;
+  if constexpr (SDT == ST_FP8) sc_in = p.scales[(u.src * p.HV + hv) * n_scale + tile];
+
+  // token prologue while the tile is in flight
+  float qv[EPL], kv[EPL];
+  ld_in_vec<EPL>(p.q, ((int64_t)b * p.H + h) * K + kofs, in_bf16, qv);
+  ld_in_vec<EPL>(p.k, ((int64_t)b * p.H + h) * K + kofs, in_bf16, kv);
+  const float v_mine = ld_in1(p.v, ((int64_t)b * p.HV + hv) * p.V + myrow_v, in_bf16);
+  const float a_in = ld_in1(p.gate, (int64_t)b * p.HV + hv, in_bf16) + p.dt_bias[hv];
+  const float b_in = ld_in1(p.beta, (int64_t)b * p.HV + hv, in_bf16);
+  const float alpha = decay_of(expf(p.A_log[hv]), a_in);
+  const float beta = (p.flags & F_BETA_PROB) ? b_in : sigmoid_f(b_in);
+  float sq = 0.f, sk = 0.f, sqk = 0.f;
+#pragma unroll
+  for (int e = 0; e < EPL; ++e) {
+    sq = fmaf(qv[e], qv[e], sq);
+    sk = fmaf(kv[e], kv[e], sk);
+    sqk = fmaf(qv[e], kv[e], sqk);
+  }
+  sq = group_sum<LPR>(sq);
+  sk = group_sum<LPR>(sk);
+  sqk = group_sum<LPR>(sqk);
+  float iq = p.scale, ik = 1.0f;
+  if (p.flags & F_L2NORM) {
+    iq *= rsqrtf(sq + kL2Eps);
+    ik = rsqrtf(sk + kL2Eps);
+  }
+  const float qk = sqk * iq * ik;
+
+  // partial k.S and q.S of every row (raw q, k)
+  float S[NR][EPL];
+  float x[NV];
+#pragma unroll
+  for (int jj = 0; jj < NR; ++jj) {
+    decode16<SDT>(raw[jj], S[jj]);
+    if constexpr (SDT == ST_FP8) {
+      const float2 sc2 = make_float2(sc_in, sc_in);
+#pragma unroll
+      for (int e = 0; e < EPL; e += 2) {
+        const float2 y = __fmul2_rn(make_float2(S[jj][e], S[jj][e + 1]), sc2);
+        S[jj][e] = y.x;
+        S[jj][e + 1] = y.y;
+      }
+    }
+    float2 ak = make_float2(0.f, 0.f), aq = make_float2(0.f, 0.f);
+#pragma unroll
+    for (int e = 0; e < EPL; e += 2) {
+      const float2 s2 = make_float2(S[jj][e], S[jj][e + 1]);
+      ak = __ffma2_rn(make_float2(kv[e], kv[e + 1]), s2, ak);
+      aq = __ffma2_rn(make_float2(qv[e], qv[e + 1]), s2, aq);
+    }
+    x[2 * jj] = ak.x + ak.y;
+    x[2 * jj + 1] = aq.x + aq.y;
+  }
+  const float mine = ReduceScatter<NV, LPR / 2>::run(x, li);
+  const float other = __shfl_xor_sync(kFull, mine, REP);
+  const float dk = (holds_q ? other : mine) * ik;
+  const float dq = (holds_q ? mine : other) * iq;
+  const float u_mine = beta * (v_mine - alpha * dk);
+  float o_mine = fmaf(qk, u_mine, alpha * dq);
+
+  // S' = alpha S + k^ u^T (u of each row from the lane that finished it)
+  float kh[EPL];
+#pragma unroll
+  for (int e = 0; e < EPL; ++e) kh[e] = kv[e] * ik;
+  const float2 al2 = make_float2(alpha, alpha);
+#pragma unroll
+  for (int jj = 0; jj < NR; ++jj) {
+    const float uj = __shfl_sync(kFull, u_mine, grp + 2 * jj * REP);
+    const float2 u2 = make_float2(uj, uj);
+#pragma unroll
+    for (int e = 0; e < EPL; e += 2) {
+      const float2 y = __ffma2_rn(make_float2(kh[e], kh[e + 1]), u2, __fmul2_rn(al2, make_float2(S[jj][e], S[jj][e + 1])));
+      S[jj][e] = y.x;
+      S[jj][e + 1] = y.y;
+    }
+  }
+
+  // storage format and store
+  char* dst = reinterpret_cast<char*>(p.pool) +
+              ((u.dst * p.HV + hv) * head_elems + (int64_t)row0 * K + kofs) * ST::BYTES;
+  const bool stored_readout = (p.flags & F_READOUT_STORED) != 0;
+  if constexpr (SDT == ST_FP8) {
+    float m = 0.f;
+#pragma unroll
+    for (int jj = 0; jj < NR; ++jj)
+#pragma unroll
+      for (int e = 0; e < EPL; ++e) m = fmaxf(m, fabsf(S[jj][e]));
+    m = group_max<32>(m);
+    if (lane == 0) s_amax[warp] = m;
+    __syncthreads();
+    float amax = s_amax[0];
+#pragma unroll
+    for (int w = 1; w < NW; ++w) amax = fmaxf(amax, s_amax[w]);
+    float sn, r;
+    fp8_scale_of(amax, sn, r);
+    const float2 r2 = make_float2(r, r);
+#pragma unroll
+    for (int jj = 0; jj < NR; ++jj) {
+      float y[EPL];
+#pragma unroll
+      for (int e = 0; e < EPL; e += 2) {
+        const float2 t = __fmul2_rn(make_float2(S[jj][e], S[jj][e + 1]), r2);
+        y[e] = t.x;
+        y[e + 1] = t.y;
+      }
+      // a zero tile (r == 0) stores +0 codes (no -0 from negative inputs)
+      const uint4 c = (r == 0.0f) ? make_uint4(0u, 0u, 0u, 0u) : encode16<SDT>(y);
+      st_stream16(dst + (int64_t)jj * RPW * K * ST::BYTES, c);
+      if (stored_readout) {
+        decode16<SDT>(c, S[jj]);
+#pragma unroll
+        for (int e = 0; e < EPL; ++e) S[jj][e] = __fmul_rn(S[jj][e], sn);
+      }
+    }
+    if (threadIdx.x == 0) p.scales[(u.dst * p.HV + hv) * n_scale + tile] = sn;
+  } else {
+#pragma unroll
+    for (int jj = 0; jj < NR; ++jj) {
+      if constexpr (SDT == ST_BF16) {
+#pragma unroll
+        for (int e = 0; e < EPL; ++e) S[jj][e] = round_bf16(S[jj][e]);
+      }
+      st_stream16(dst + (int64_t)jj * RPW * K * ST::BYTES, encode16<SDT>(S[jj]));
+    }
+  }
+  if constexpr (SDT != ST_F32) {
+    if (stored_readout) {
+      // o from the stored state: q^.S' of every row through the same reduction
+#pragma unroll
+      for (int jj = 0; jj < NR; ++jj) {
+        float y = 0.f;
+#pragma unroll
+        for (int e = 0; e < EPL; ++e) y = fmaf(qv[e], S[jj][e], y);
+        x[2 * jj] = y * iq;
+        x[2 * jj + 1] = 0.f;
+      }
+      o_mine = ReduceScatter<NV, LPR / 2>::run(x, li);
+    }
+  }
+  if (writer) st_out1(p.out, out_at, o_mine, (p.flags & F_OUT_BF16) != 0);
+}
+
+}  // namespace gdn

@@ -23,6 +23,13 @@ from oracle import gdn as O
 
 TOL = {"f32": 1e-4, "bf16": 2e-2, "fp8_e4m3": 1e-4}
 BF16_OUT = 2.0 ** -8
+# fp8 state read out from the STORED (re-encoded) state: where the two fp32
+# working states straddle an E4M3 rounding boundary the two sides store
+# neighbouring codes, and o moves by |q_i| times one E4M3 step (at most
+# 2^-3 of the element's magnitude). With unit-norm q scaled by 1/sqrt(K) and
+# a handful of such codes per tile, 1e-2 of the slice's max bounds it; the
+# output is then also checked against the stored state it was read from.
+TOL_FP8_STORED = 1e-2
 
 
 def dev(x: np.ndarray, dtype=None):
@@ -117,6 +124,23 @@ def check_untouched(pool_before: np.ndarray, pool_after: np.ndarray, written_key
         assert np.array_equal(scales_before[mask].view(np.uint32), scales_after[mask].view(np.uint32))
 
 
+def check_stored_readout(out_gpu, t, idx, pool_after, scales_after, units, layout, scale, use_qk_l2norm,
+                         num_slots, block_v=64):
+    """Validity of a stored readout: the last token's output is q^ times the
+    state the kernel stored (decoded by the oracle's codec)."""
+    K = t["q"].shape[-1]
+    H, HV = t["q"].shape[2], t["v"].shape[2]
+    sc = O._scale_of(scale, K)
+    for (b, hv) in units:
+        s = int(idx[b])
+        if not 0 <= s < num_slots:
+            continue
+        qh, _ = O.prepare_qk(t["q"][b, -1, O.key_head_of(hv, H, HV)], t["k"][b, -1, 0], sc, use_qk_l2norm)
+        S = O.load_state(pool_after[s, hv], layout, "fp8_e4m3", scales_after[s, hv], block_v)
+        e = slice_rel_err(out_gpu[b, -1, hv], qh @ S)
+        assert e <= 1e-4, f"stored readout (b={b}, hv={hv}) is not q^T of the stored state: {e:.3g}"
+
+
 # ----------------------------------------------------------------------------
 # GDN slot pool case
 # ----------------------------------------------------------------------------
@@ -154,8 +178,12 @@ def gdn_slots_case(seed, B, T, H, HV, K, V, num_slots, layout="V_FIRST", state_d
         scale=scale, use_qk_l2norm=use_qk_l2norm, readout_mode=readout, num_slots=num_slots,
         units=units)
     todo = [(b, hv) for b in range(B) for hv in range(HV)] if units is None else units
+    tol = TOL_FP8_STORED if (state_dtype == "fp8_e4m3" and readout == "stored") else TOL[state_dtype]
     res["out_err"] = check_outputs(res["out"], ref_out, todo, lambda x, b, hv: x[b, :, hv, :],
-                                   TOL[state_dtype], out_dtype)
+                                   tol, out_dtype)
+    if state_dtype == "fp8_e4m3" and readout == "stored":
+        check_stored_readout(res["out"], t, idx, after, sc_after, todo, layout, scale, use_qk_l2norm,
+                             num_slots, block_v)
     res["state_err"] = check_state(after, sc_after, writes, state_dtype, layout, block_v)
     written = {(s, hv) for s in live for hv in range(HV)} if T > 0 else set()
     check_untouched(before, after, written, sc_before, sc_after)
