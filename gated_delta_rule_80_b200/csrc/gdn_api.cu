@@ -80,9 +80,10 @@ template <int SDT, int K, int IDX>
 int launch_tile1(StepParams p, int B, cudaStream_t s) {
   using TS = Tile1Shape<SDT, K>;
   p.n_vtiles = p.V / TS::VT;
-  const int64_t units = static_cast<int64_t>(B) * p.HV * p.n_vtiles;
-  if (units > INT_MAX) return GDN_ERR_INVALID_ARG;
-  step_tile1<SDT, K, IDX><<<static_cast<unsigned>(units), TS::NW * 32, 0, s>>>(p);
+  p.G = p.HV / p.H;
+  if (B > 65535) return GDN_ERR_INVALID_ARG;  // grid z
+  const dim3 grid(p.n_vtiles, p.HV, B);
+  step_tile1<SDT, K, IDX><<<grid, TS::NW * 32, 0, s>>>(p);
   return launch_status();
 }
 

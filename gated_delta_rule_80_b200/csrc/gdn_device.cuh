@@ -58,6 +58,7 @@ struct StepParams {
   int64_t num_slots;
   int64_t nnz;
   int B, T, H, HV, V;
+  int G;                // value heads per key head, HV / H
   int n_vtiles;
   int total_tokens;
   int page_size;
@@ -144,6 +145,27 @@ __device__ __forceinline__ uint4 encode16(const float* x) {
     }
   }
   return make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+// 8 stored fp8 bytes <-> 8 floats (codes unscaled)
+__device__ __forceinline__ void decode8_fp8(uint2 raw, float* x) {
+  const uint32_t w[2] = {raw.x, raw.y};
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    float2 a = e4m3x2_to_float2(static_cast<uint16_t>(w[i] & 0xffffu));
+    float2 b = e4m3x2_to_float2(static_cast<uint16_t>(w[i] >> 16));
+    x[4 * i] = a.x; x[4 * i + 1] = a.y; x[4 * i + 2] = b.x; x[4 * i + 3] = b.y;
+  }
+}
+__device__ __forceinline__ uint2 encode8_fp8(const float* x) {
+  uint32_t w[2];
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    uint32_t lo = float2_to_e4m3x2(x[4 * i], x[4 * i + 1]);
+    uint32_t hi = float2_to_e4m3x2(x[4 * i + 2], x[4 * i + 3]);
+    w[i] = lo | (hi << 16);
+  }
+  return make_uint2(w[0], w[1]);
 }
 
 // fp8 tile scale from the tile's amax: s = amax / 448 and r = 1 / s, both

@@ -27,7 +27,32 @@ namespace gdn {
 template <int SDT, int K>
 struct Tile1Shape {
   static constexpr int VT = (SDT == ST_FP8) ? 64 : 32;   // fp8: the [K, 64] scale tile
-  static constexpr int NW = (SDT == ST_FP8 && K > 32) ? 8 : 4;
+  static constexpr int NW = (SDT == ST_FP8) ? 8 : 4;
+  // bytes one lane moves per row: 16, except 8 for fp8 (keeps q/k per lane small)
+  static constexpr int VB = (SDT == ST_FP8) ? 8 : 16;
+  // resident CTAs per SM the register budget is sized for
+  static constexpr int MIN_CTAS = (SDT == ST_FP8) ? 3 : 8;
+};
+
+// Vector of VB stored bytes: load/store and decode/encode.
+template <int SDT, int VB> struct StateVec;
+template <int SDT> struct StateVec<SDT, 16> {
+  using T = uint4;
+  static constexpr int EPL = StateTraits<SDT>::EPL;
+  __device__ __forceinline__ static T load(const char* p) { return ld_stream16(p); }
+  __device__ __forceinline__ static void store(char* p, T v) { st_stream16(p, v); }
+  __device__ __forceinline__ static void decode(T v, float* x) { decode16<SDT>(v, x); }
+  __device__ __forceinline__ static T encode(const float* x) { return encode16<SDT>(x); }
+  __device__ __forceinline__ static T zero() { return make_uint4(0u, 0u, 0u, 0u); }
+};
+template <> struct StateVec<ST_FP8, 8> {
+  using T = uint2;
+  static constexpr int EPL = 8;
+  __device__ __forceinline__ static T load(const char* p) { return __ldcs(reinterpret_cast<const uint2*>(p)); }
+  __device__ __forceinline__ static void store(char* p, T v) { __stcs(reinterpret_cast<uint2*>(p), v); }
+  __device__ __forceinline__ static void decode(T v, float* x) { decode8_fp8(v, x); }
+  __device__ __forceinline__ static T encode(const float* x) { return encode8_fp8(x); }
+  __device__ __forceinline__ static T zero() { return make_uint2(0u, 0u); }
 };
 
 // Reduce-scatter of N values over the lanes of a row group: each halving
@@ -57,21 +82,25 @@ struct ReduceScatter {
 };
 
 template <int SDT, int K, int IDX>
-__global__ void __launch_bounds__(Tile1Shape<SDT, K>::NW * 32)
+__global__ void __launch_bounds__(Tile1Shape<SDT, K>::NW * 32, Tile1Shape<SDT, K>::MIN_CTAS)
 step_tile1(const StepParams p) {
   using ST = StateTraits<SDT>;
-  constexpr int EPL = ST::EPL;
+  using TS = Tile1Shape<SDT, K>;
+  using SV = StateVec<SDT, TS::VB>;
+  constexpr int EPL = SV::EPL;
   constexpr int LPR = K / EPL;  // lanes per stored row
   static_assert(K % EPL == 0 && LPR >= 2 && LPR <= 32 && 32 % LPR == 0, "row must fit a warp");
   constexpr int RPW = 32 / LPR;  // rows per warp instruction
-  constexpr int VT = Tile1Shape<SDT, K>::VT;
-  constexpr int NW = Tile1Shape<SDT, K>::NW;
+  constexpr int VT = TS::VT;
+  constexpr int NW = TS::NW;
   constexpr int NR = VT / (NW * RPW);  // rows per thread
   static_assert(NR >= 1 && NR * NW * RPW == VT, "tile must split evenly");
   constexpr int NV = 2 * NR;           // k.S and q.S partial sums per thread
   static_assert(NV <= LPR, "one finished sum per lane");
   constexpr int REP = LPR / NV;        // lanes that end with the same sum
+  constexpr int ROWB = K * ST::BYTES;  // bytes of one stored row
 
+  __shared__ float s_pro[5];           // alpha, beta, q scale, k scale, q^.k^
   __shared__ float s_amax[NW];
 
   const int lane = threadIdx.x & 31;
@@ -83,12 +112,10 @@ step_tile1(const StepParams p) {
   const bool holds_q = (vidx & 1) != 0;
   const int grp = lane - li;
   const bool writer = !holds_q && (li % REP) == 0;
-  int unit = blockIdx.x;
-  const int tile = unit % p.n_vtiles;
-  unit /= p.n_vtiles;
-  const int hv = unit % p.HV;
-  const int b = unit / p.HV;           // T == 1: the token of sequence b is b
-  const int h = hv / (p.HV / p.H);
+  const int tile = blockIdx.x;
+  const int hv = blockIdx.y;
+  const int b = blockIdx.z;            // T == 1: the token of sequence b is b
+  const int h = hv / p.G;
   const int kofs = li * EPL;
   const bool in_bf16 = (p.flags & F_IN_BF16) != 0;
   const int row0 = tile * VT + warp * NR * RPW + ri;   // row jj is row0 + jj * RPW
@@ -104,57 +131,61 @@ step_tile1(const StepParams p) {
   }
 
   // all state loads first
-  const int64_t head_elems = (int64_t)K * p.V;
-  const char* src = reinterpret_cast<const char*>(p.pool) +
-                    ((u.src * p.HV + hv) * head_elems + (int64_t)row0 * K + kofs) * ST::BYTES;
-  uint4 raw[NR];
+  const int64_t head_bytes = (int64_t)K * p.V * ST::BYTES;
+  const char* src = reinterpret_cast<const char*>(p.pool) + (u.src * p.HV + hv) * head_bytes +
+                    (int64_t)row0 * ROWB + kofs * ST::BYTES;
+  typename SV::T raw[NR];
 #pragma unroll
-  for (int jj = 0; jj < NR; ++jj) raw[jj] = ld_stream16(src + (int64_t)jj * RPW * K * ST::BYTES);
+  for (int jj = 0; jj < NR; ++jj) raw[jj] = SV::load(src + jj * RPW * ROWB);
   [[maybe_unused]] float sc_in = 1.0f;
   const int n_scale = p.V / VT;
   if constexpr (SDT == ST_FP8) sc_in = p.scales[(u.src * p.HV + hv) * n_scale + tile];
 
-  // token prologue while the tile is in flight
+  // token prologue while the tile is in flight: warp 0 computes the
+  // per-token scalars, every lane loads its own q/k/v entries
   float qv[EPL], kv[EPL];
   ld_in_vec<EPL>(p.q, ((int64_t)b * p.H + h) * K + kofs, in_bf16, qv);
   ld_in_vec<EPL>(p.k, ((int64_t)b * p.H + h) * K + kofs, in_bf16, kv);
   const float v_mine = ld_in1(p.v, ((int64_t)b * p.HV + hv) * p.V + myrow_v, in_bf16);
-  const float a_in = ld_in1(p.gate, (int64_t)b * p.HV + hv, in_bf16) + p.dt_bias[hv];
-  const float b_in = ld_in1(p.beta, (int64_t)b * p.HV + hv, in_bf16);
-  const float alpha = decay_of(expf(p.A_log[hv]), a_in);
-  const float beta = (p.flags & F_BETA_PROB) ? b_in : sigmoid_f(b_in);
-  float sq = 0.f, sk = 0.f, sqk = 0.f;
+  if (warp == 0) {
+    constexpr int KPL = K / 32;
+    float qn[KPL], kn[KPL];
+    ld_in_vec<KPL>(p.q, ((int64_t)b * p.H + h) * K + lane * KPL, in_bf16, qn);
+    ld_in_vec<KPL>(p.k, ((int64_t)b * p.H + h) * K + lane * KPL, in_bf16, kn);
+    float sq = 0.f, sk = 0.f, sqk = 0.f;
 #pragma unroll
-  for (int e = 0; e < EPL; ++e) {
-    sq = fmaf(qv[e], qv[e], sq);
-    sk = fmaf(kv[e], kv[e], sk);
-    sqk = fmaf(qv[e], kv[e], sqk);
+    for (int e = 0; e < KPL; ++e) {
+      sq = fmaf(qn[e], qn[e], sq);
+      sk = fmaf(kn[e], kn[e], sk);
+      sqk = fmaf(qn[e], kn[e], sqk);
+    }
+    sq = group_sum<32>(sq);
+    sk = group_sum<32>(sk);
+    sqk = group_sum<32>(sqk);
+    if (lane == 0) {
+      float iq = p.scale, ik = 1.0f;
+      if (p.flags & F_L2NORM) {
+        iq *= rsqrtf(sq + kL2Eps);
+        ik = rsqrtf(sk + kL2Eps);
+      }
+      const float a_in = ld_in1(p.gate, (int64_t)b * p.HV + hv, in_bf16) + p.dt_bias[hv];
+      const float b_in = ld_in1(p.beta, (int64_t)b * p.HV + hv, in_bf16);
+      s_pro[0] = decay_of(expf(p.A_log[hv]), a_in);
+      s_pro[1] = (p.flags & F_BETA_PROB) ? b_in : sigmoid_f(b_in);
+      s_pro[2] = iq;
+      s_pro[3] = ik;
+      s_pro[4] = sqk * iq * ik;
+    }
   }
-  sq = group_sum<LPR>(sq);
-  sk = group_sum<LPR>(sk);
-  sqk = group_sum<LPR>(sqk);
-  float iq = p.scale, ik = 1.0f;
-  if (p.flags & F_L2NORM) {
-    iq *= rsqrtf(sq + kL2Eps);
-    ik = rsqrtf(sk + kL2Eps);
-  }
-  const float qk = sqk * iq * ik;
+  __syncthreads();
+  const float alpha = s_pro[0], beta = s_pro[1], iq = s_pro[2], ik = s_pro[3], qk = s_pro[4];
 
-  // partial k.S and q.S of every row (raw q, k)
+  // partial k.S and q.S of every row (raw q, k; fp8: raw code values)
   float S[NR][EPL];
   float x[NV];
 #pragma unroll
   for (int jj = 0; jj < NR; ++jj) {
-    decode16<SDT>(raw[jj], S[jj]);
-    if constexpr (SDT == ST_FP8) {
-      const float2 sc2 = make_float2(sc_in, sc_in);
-#pragma unroll
-      for (int e = 0; e < EPL; e += 2) {
-        const float2 y = __fmul2_rn(make_float2(S[jj][e], S[jj][e + 1]), sc2);
-        S[jj][e] = y.x;
-        S[jj][e + 1] = y.y;
-      }
-    }
+    SV::decode(raw[jj], S[jj]);
     float2 ak = make_float2(0.f, 0.f), aq = make_float2(0.f, 0.f);
 #pragma unroll
     for (int e = 0; e < EPL; e += 2) {
@@ -167,31 +198,33 @@ step_tile1(const StepParams p) {
   }
   const float mine = ReduceScatter<NV, LPR / 2>::run(x, li);
   const float other = __shfl_xor_sync(kFull, mine, REP);
-  const float dk = (holds_q ? other : mine) * ik;
-  const float dq = (holds_q ? mine : other) * iq;
+  const float dk = (holds_q ? other : mine) * (ik * sc_in);
+  const float dq = (holds_q ? mine : other) * (iq * sc_in);
   const float u_mine = beta * (v_mine - alpha * dk);
   float o_mine = fmaf(qk, u_mine, alpha * dq);
 
-  // S' = alpha S + k^ u^T (u of each row from the lane that finished it)
+  // S' = alpha S + k^ u^T (u of each row from the lane that finished it);
+  // fp8: S holds code values, so the decay factor carries the tile scale
   float kh[EPL];
 #pragma unroll
   for (int e = 0; e < EPL; ++e) kh[e] = kv[e] * ik;
-  const float2 al2 = make_float2(alpha, alpha);
+  const float f = (SDT == ST_FP8) ? __fmul_rn(alpha, sc_in) : alpha;
+  const float2 f2 = make_float2(f, f);
 #pragma unroll
   for (int jj = 0; jj < NR; ++jj) {
     const float uj = __shfl_sync(kFull, u_mine, grp + 2 * jj * REP);
     const float2 u2 = make_float2(uj, uj);
 #pragma unroll
     for (int e = 0; e < EPL; e += 2) {
-      const float2 y = __ffma2_rn(make_float2(kh[e], kh[e + 1]), u2, __fmul2_rn(al2, make_float2(S[jj][e], S[jj][e + 1])));
+      const float2 y = __ffma2_rn(make_float2(kh[e], kh[e + 1]), u2, __fmul2_rn(f2, make_float2(S[jj][e], S[jj][e + 1])));
       S[jj][e] = y.x;
       S[jj][e + 1] = y.y;
     }
   }
 
   // storage format and store
-  char* dst = reinterpret_cast<char*>(p.pool) +
-              ((u.dst * p.HV + hv) * head_elems + (int64_t)row0 * K + kofs) * ST::BYTES;
+  char* dst = reinterpret_cast<char*>(p.pool) + (u.dst * p.HV + hv) * head_bytes + (int64_t)row0 * ROWB +
+              kofs * ST::BYTES;
   const bool stored_readout = (p.flags & F_READOUT_STORED) != 0;
   if constexpr (SDT == ST_FP8) {
     float m = 0.f;
@@ -218,10 +251,10 @@ step_tile1(const StepParams p) {
         y[e + 1] = t.y;
       }
       // a zero tile (r == 0) stores +0 codes (no -0 from negative inputs)
-      const uint4 c = (r == 0.0f) ? make_uint4(0u, 0u, 0u, 0u) : encode16<SDT>(y);
-      st_stream16(dst + (int64_t)jj * RPW * K * ST::BYTES, c);
+      const typename SV::T c = (r == 0.0f) ? SV::zero() : SV::encode(y);
+      SV::store(dst + jj * RPW * ROWB, c);
       if (stored_readout) {
-        decode16<SDT>(c, S[jj]);
+        SV::decode(c, S[jj]);
 #pragma unroll
         for (int e = 0; e < EPL; ++e) S[jj][e] = __fmul_rn(S[jj][e], sn);
       }
@@ -234,7 +267,7 @@ step_tile1(const StepParams p) {
 #pragma unroll
         for (int e = 0; e < EPL; ++e) S[jj][e] = round_bf16(S[jj][e]);
       }
-      st_stream16(dst + (int64_t)jj * RPW * K * ST::BYTES, encode16<SDT>(S[jj]));
+      SV::store(dst + jj * RPW * ROWB, SV::encode(S[jj]));
     }
   }
   if constexpr (SDT != ST_F32) {
