@@ -178,9 +178,9 @@ __global__ void __launch_bounds__(128) fp8_quantize_kernel(const float* src, uin
       x[i][4 * c] = f.x; x[i][4 * c + 1] = f.y; x[i][4 * c + 2] = f.z; x[i][4 * c + 3] = f.w;
     }
 #pragma unroll
-    for (int e = 0; e < 16; ++e) m = fmaxf(m, fabsf(x[i][e]));
+    for (int e = 0; e < 16; ++e) m = absmax_acc(m, x[i][e]);
   }
-  m = group_max<32>(m);
+  m = group_max<32>(fabsf(m));
   if ((threadIdx.x & 31) == 0) s_amax[threadIdx.x >> 5] = m;
   __syncthreads();
   float amax = s_amax[0];

@@ -168,6 +168,15 @@ __device__ __forceinline__ uint2 encode8_fp8(const float* x) {
   return make_uint2(w[0], w[1]);
 }
 
+// Running max of |x|: max.xorsign.abs gives max(|m|, |x|) (with the xor of
+// the signs, which the caller drops with one fabsf at the end), one
+// instruction per element instead of an abs and a max.
+__device__ __forceinline__ float absmax_acc(float m, float x) {
+  float r;
+  asm("max.xorsign.abs.f32 %0, %1, %2;" : "=f"(r) : "f"(m), "f"(x));
+  return r;
+}
+
 // fp8 tile scale from the tile's amax: s = amax / 448 and r = 1 / s, both
 // correctly rounded; a zero tile (or one whose r overflows) stores s = 0 and
 // codes 0 (signalled by r = 0).

@@ -232,8 +232,8 @@ step_vfirst(const StepParams p) {
 #pragma unroll
       for (int j = 0; j < NR; ++j)
 #pragma unroll
-        for (int e = 0; e < EPL; ++e) m = fmaxf(m, fabsf(S[j][e]));
-      m = group_max<32>(m);
+        for (int e = 0; e < EPL; ++e) m = absmax_acc(m, S[j][e]);
+      m = group_max<32>(fabsf(m));
       const int buf = (tok - u.tok0) & 1;
       if (lane == 0) s_amax[buf][warp] = m;
       __syncthreads();
@@ -473,8 +473,8 @@ step_kfirst(const StepParams p) {
 #pragma unroll
       for (int j = 0; j < KR; ++j)
 #pragma unroll
-        for (int e = 0; e < EPL; ++e) m = fmaxf(m, fabsf(S[j][e]));
-      m = group_max<32>(m);
+        for (int e = 0; e < EPL; ++e) m = absmax_acc(m, S[j][e]);
+      m = group_max<32>(fabsf(m));
       if (lane == 0) s_amax[buf][warp] = m;
       __syncthreads();
       float amax = s_amax[buf][0];

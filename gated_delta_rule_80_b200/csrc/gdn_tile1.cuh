@@ -27,11 +27,12 @@ namespace gdn {
 template <int SDT, int K>
 struct Tile1Shape {
   static constexpr int VT = (SDT == ST_FP8) ? 64 : 32;   // fp8: the [K, 64] scale tile
-  static constexpr int NW = (SDT == ST_FP8) ? 8 : 4;
-  // bytes one lane moves per row: 16, except 8 for fp8 (keeps q/k per lane small)
-  static constexpr int VB = (SDT == ST_FP8) ? 8 : 16;
-  // resident CTAs per SM the register budget is sized for
-  static constexpr int MIN_CTAS = (SDT == ST_FP8) ? 3 : 8;
+  static constexpr int NW = 4;
+  // bytes one lane moves per row
+  static constexpr int VB = 16;
+  // resident CTAs per SM the register budget is sized for (fp8 holds 64
+  // decoded elements per thread)
+  static constexpr int MIN_CTAS = (SDT == ST_FP8) ? 4 : 8;
 };
 
 // Vector of VB stored bytes: load/store and decode/encode.
@@ -231,8 +232,8 @@ step_tile1(const StepParams p) {
 #pragma unroll
     for (int jj = 0; jj < NR; ++jj)
 #pragma unroll
-      for (int e = 0; e < EPL; ++e) m = fmaxf(m, fabsf(S[jj][e]));
-    m = group_max<32>(m);
+      for (int e = 0; e < EPL; ++e) m = absmax_acc(m, S[jj][e]);
+    m = group_max<32>(fabsf(m));
     if (lane == 0) s_amax[warp] = m;
     __syncthreads();
     float amax = s_amax[0];
@@ -241,22 +242,31 @@ step_tile1(const StepParams p) {
     float sn, r;
     fp8_scale_of(amax, sn, r);
     const float2 r2 = make_float2(r, r);
+    if (r != 0.0f) {
 #pragma unroll
-    for (int jj = 0; jj < NR; ++jj) {
-      float y[EPL];
+      for (int jj = 0; jj < NR; ++jj) {
+        float y[EPL];
 #pragma unroll
-      for (int e = 0; e < EPL; e += 2) {
-        const float2 t = __fmul2_rn(make_float2(S[jj][e], S[jj][e + 1]), r2);
-        y[e] = t.x;
-        y[e + 1] = t.y;
+        for (int e = 0; e < EPL; e += 2) {
+          const float2 t = __fmul2_rn(make_float2(S[jj][e], S[jj][e + 1]), r2);
+          y[e] = t.x;
+          y[e + 1] = t.y;
+        }
+        const typename SV::T c = SV::encode(y);
+        SV::store(dst + jj * RPW * ROWB, c);
+        if (stored_readout) {
+          SV::decode(c, S[jj]);
+#pragma unroll
+          for (int e = 0; e < EPL; ++e) S[jj][e] = __fmul_rn(S[jj][e], sn);
+        }
       }
-      // a zero tile (r == 0) stores +0 codes (no -0 from negative inputs)
-      const typename SV::T c = (r == 0.0f) ? SV::zero() : SV::encode(y);
-      SV::store(dst + jj * RPW * ROWB, c);
-      if (stored_readout) {
-        SV::decode(c, S[jj]);
+    } else {
+      // a zero tile stores +0 codes (no -0 from negative inputs)
 #pragma unroll
-        for (int e = 0; e < EPL; ++e) S[jj][e] = __fmul_rn(S[jj][e], sn);
+      for (int jj = 0; jj < NR; ++jj) {
+        SV::store(dst + jj * RPW * ROWB, SV::zero());
+#pragma unroll
+        for (int e = 0; e < EPL; ++e) S[jj][e] = 0.0f;
       }
     }
     if (threadIdx.x == 0) p.scales[(u.dst * p.HV + hv) * n_scale + tile] = sn;
