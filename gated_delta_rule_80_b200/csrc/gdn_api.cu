@@ -13,7 +13,7 @@
 #include <utility>
 
 #include "../../include/gdn.h"
-#include "gdn_tile1.cuh"
+#include "gdn_seq.cuh"
 
 using namespace gdn;
 
@@ -80,26 +80,33 @@ template <int SDT, int K, int IDX>
 int launch_tile1(StepParams p, int B, cudaStream_t s) {
   using TS = Tile1Shape<SDT, K>;
   p.n_vtiles = p.V / TS::VT;
-  p.G = p.HV / p.H;
-  if (B > 65535) return GDN_ERR_INVALID_ARG;  // grid z
   const dim3 grid(p.n_vtiles, p.HV, B);
   step_tile1<SDT, K, IDX><<<grid, TS::NW * 32, 0, s>>>(p);
   return launch_status();
 }
 
+// T >= 1 tokens per unit, either layout: the chunked-prologue kernel.
+template <int L, int SDT, int K, int GATE, int IDX, int NW>
+int launch_seq_nw(StepParams p, int B, cudaStream_t s) {
+  using SH = SeqShape<SDT, L, K, NW>;
+  p.n_vtiles = p.V / SH::VC;
+  const dim3 grid(p.n_vtiles, p.HV, B);
+  step_seq<SDT, L, K, GATE, IDX, NW><<<grid, NW * 32, 0, s>>>(p);
+  return launch_status();
+}
+
 template <int L, int SDT, int K, int GATE, int IDX>
 int launch_one(StepParams p, int B, cudaStream_t s) {
+  p.G = p.HV / p.H;
+  if (B > 65535) return GDN_ERR_INVALID_ARG;  // grid z
   if constexpr (L == L_VFIRST && GATE == GATE_SCALAR) {
     if (p.T == 1) return launch_tile1<SDT, K, IDX>(p, B, s);
   }
-  constexpr int VT = TileShape<SDT>::VT;
-  constexpr int NT = TileShape<SDT>::NW * 32;
-  p.n_vtiles = p.V / VT;
-  const int64_t units = static_cast<int64_t>(B) * p.HV * p.n_vtiles;
-  if (units > INT_MAX) return GDN_ERR_INVALID_ARG;
-  if constexpr (L == L_VFIRST) step_vfirst<SDT, K, GATE, IDX><<<static_cast<unsigned>(units), NT, 0, s>>>(p);
-  else step_kfirst<SDT, K, GATE, IDX><<<static_cast<unsigned>(units), NT, 0, s>>>(p);
-  return launch_status();
+  if constexpr (L == L_KFIRST && SDT != ST_FP8) {
+    // 16 columns per warp: 4 warps when V allows a 64-column tile
+    if (p.V % 64 != 0) return launch_seq_nw<L, SDT, K, GATE, IDX, 2>(p, B, s);
+  }
+  return launch_seq_nw<L, SDT, K, GATE, IDX, 4>(p, B, s);
 }
 
 template <int L, int SDT, int GATE, int IDX>

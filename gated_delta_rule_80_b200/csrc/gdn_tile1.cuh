@@ -20,7 +20,7 @@
 //     S' = alpha S + k^ u^T.
 #pragma once
 
-#include "gdn_step.cuh"
+#include "gdn_device.cuh"
 
 namespace gdn {
 
@@ -45,6 +45,19 @@ template <int SDT> struct StateVec<SDT, 16> {
   __device__ __forceinline__ static void decode(T v, float* x) { decode16<SDT>(v, x); }
   __device__ __forceinline__ static T encode(const float* x) { return encode16<SDT>(x); }
   __device__ __forceinline__ static T zero() { return make_uint4(0u, 0u, 0u, 0u); }
+};
+template <> struct StateVec<ST_BF16, 8> {
+  using T = uint2;
+  static constexpr int EPL = 4;
+  __device__ __forceinline__ static T load(const char* p) { return __ldcs(reinterpret_cast<const uint2*>(p)); }
+  __device__ __forceinline__ static void store(char* p, T v) { __stcs(reinterpret_cast<uint2*>(p), v); }
+  __device__ __forceinline__ static void decode(T v, float* x) {
+    x[0] = bf16_lo(v.x); x[1] = bf16_hi(v.x); x[2] = bf16_lo(v.y); x[3] = bf16_hi(v.y);
+  }
+  __device__ __forceinline__ static T encode(const float* x) {
+    return make_uint2(pack_bf16x2(x[0], x[1]), pack_bf16x2(x[2], x[3]));
+  }
+  __device__ __forceinline__ static T zero() { return make_uint2(0u, 0u); }
 };
 template <> struct StateVec<ST_FP8, 8> {
   using T = uint2;
