@@ -75,7 +75,7 @@ class gdn_decode_slots_params(ctypes.Structure):
 
 
 class gdn_decode_paged_params(ctypes.Structure):
-    _fields_ = [("struct_size", _i32), ("B", _i32), ("H", _i32), ("HV", _i32), ("K", _i32),
+    _fields_ = [("struct_size", _i32), ("B", _i32), ("T", _i32), ("H", _i32), ("HV", _i32), ("K", _i32),
                 ("V", _i32), ("in_dtype", _i32), ("out_dtype", _i32), ("index_dtype", _i32),
                 ("readout", _i32), ("use_qk_l2norm", _i32), ("page_size", _i32),
                 ("scale", ctypes.c_float), ("nnz", _i64), ("q", _vp), ("k", _vp), ("v", _vp),
@@ -257,21 +257,25 @@ def gdn_decode_paged(q, k, v, A_log, a, dt_bias, b, scale=None, output=None, use
                      state_pool, page_indices, page_indptr, last_page_len, slots=None,
                      state_scales=None, state_layout="V_FIRST", block_v=64, page_size=0,
                      output_dtype=None, readout="working", err_flags=None):
-    """Single-token GDN decode on a paged pool [num_pages, HV, V, K].
+    """GDN decode of the last T tokens of every sequence on a paged pool
+    [num_pages, HV, V, K].
 
-    q, k [B, 1, H, K]; v [B, 1, HV, V]; a, b [B, 1, HV]; the CSR page table
-    (page_indices, page_indptr, last_page_len) in one int dtype; slots: an
-    optional int64 [B, 2] tensor of (read_page, write_page) rows from
-    ``gdn_paged_decode_slots``. Returns output [B, 1, HV, V].
+    q, k [B, T, H, K]; v [B, T, HV, V]; a, b [B, T, HV]; the CSR page table
+    (page_indices, page_indptr, last_page_len) in one int dtype; slots (T ==
+    1 only): an optional int64 [B, 2] tensor of (read_page, write_page) rows
+    from ``gdn_paged_decode_slots``. T > 1 needs page_size. Returns output
+    [B, T, HV, V].
     """
     B, T, H, K = q.shape
-    if T != 1:
-        raise ValueError("paged decode takes exactly one token per sequence")
+    if T > 1 and page_size <= 0:
+        raise ValueError("a multi-token suffix needs page_size")
+    if T > 1 and slots is not None:
+        raise ValueError("precomputed slots rows describe single-token calls only")
     HV, V = v.shape[2], v.shape[3]
-    _expect(k, (B, 1, H, K), "k")
-    _expect(v, (B, 1, HV, V), "v")
-    _expect(a, (B, 1, HV), "a")
-    _expect(b, (B, 1, HV), "b")
+    _expect(k, (B, T, H, K), "k")
+    _expect(v, (B, T, HV, V), "v")
+    _expect(a, (B, T, HV), "a")
+    _expect(b, (B, T, HV), "b")
     _expect(A_log, (HV,), "A_log")
     _expect(dt_bias, (HV,), "dt_bias")
     _expect(page_indptr, (B + 1,), "page_indptr")
@@ -283,10 +287,10 @@ def gdn_decode_paged(q, k, v, A_log, a, dt_bias, b, scale=None, output=None, use
     if len({x.dtype for x in (q, k, v, a, b)}) != 1:
         raise ValueError("q, k, v, a, b must share one dtype")
     out_dt = output_dtype or (output.dtype if output is not None else q.dtype)
-    out = _out(output, (B, 1, HV, V), out_dt, q)
+    out = _out(output, (B, T, HV, V), out_dt, q)
     prm = gdn_decode_paged_params()
     prm.struct_size = ctypes.sizeof(gdn_decode_paged_params)
-    prm.B, prm.H, prm.HV, prm.K, prm.V = B, H, HV, K, V
+    prm.B, prm.T, prm.H, prm.HV, prm.K, prm.V = B, T, H, HV, K, V
     prm.in_dtype, prm.out_dtype = _io_dtype(q), _io_dtype(out)
     prm.index_dtype = _same_index_dtype(page_indices, page_indptr, last_page_len)
     prm.readout = _READOUTS[readout]

@@ -292,13 +292,16 @@ int gdn_decode_slots(const gdn_decode_slots_params* p, gdn_stream_t stream) {
 int gdn_decode_paged(const gdn_decode_paged_params* p, gdn_stream_t stream) {
   if (p == nullptr || p->struct_size != static_cast<int32_t>(sizeof(gdn_decode_paged_params)))
     return GDN_ERR_INVALID_ARG;
-  if (p->B < 0 || p->H <= 0 || p->HV <= 0 || p->HV % p->H != 0 || p->nnz < 0) return GDN_ERR_INVALID_ARG;
+  if (p->B < 0 || p->T < 0 || p->H <= 0 || p->HV <= 0 || p->HV % p->H != 0 || p->nnz < 0)
+    return GDN_ERR_INVALID_ARG;
+  if (p->T > 1 && (p->page_size <= 0 || p->slots != nullptr)) return GDN_ERR_INVALID_ARG;
+  if (static_cast<int64_t>(p->B) * p->T > INT_MAX) return GDN_ERR_INVALID_ARG;
   if (!head_dim_ok(p->K) || !head_dim_ok(p->V)) return GDN_ERR_INVALID_ARG;
   if (!io_dtype_ok(p->in_dtype) || !io_dtype_ok(p->out_dtype)) return GDN_ERR_INVALID_ARG;
   if (p->index_dtype != GDN_I32 && p->index_dtype != GDN_I64) return GDN_ERR_INVALID_ARG;
   if (p->readout != GDN_READOUT_WORKING && p->readout != GDN_READOUT_STORED) return GDN_ERR_INVALID_ARG;
   if (const int rc = check_pool(p->pool, p->V)) return rc;
-  if (p->B == 0) return GDN_OK;
+  if (p->B == 0 || p->T == 0) return GDN_OK;
   const uintptr_t es = io_size(p->in_dtype), is = index_size(p->index_dtype);
   if (!ptrs_ok({p->q, p->k, p->v, p->out}, {{p->a, es}, {p->b, es}, {p->A_log, 4}, {p->dt_bias, 4}}))
     return GDN_ERR_INVALID_ARG;
@@ -317,8 +320,8 @@ int gdn_decode_paged(const gdn_decode_paged_params* p, gdn_stream_t stream) {
   k.idx = p->page_indices; k.indptr = p->page_indptr; k.lastlen = p->last_page_len; k.rows = p->slots;
   k.out = p->out; k.err = p->err_flags;
   k.num_slots = p->pool.num_slots; k.nnz = p->nnz;
-  k.B = p->B; k.T = 1; k.H = p->H; k.HV = p->HV; k.V = p->V;
-  k.total_tokens = p->B;
+  k.B = p->B; k.T = p->T; k.H = p->H; k.HV = p->HV; k.V = p->V;
+  k.total_tokens = p->B * p->T;
   k.page_size = p->page_size;
   k.scale = default_scale(p->scale, p->K);
   k.flags = (p->in_dtype == GDN_BF16 ? F_IN_BF16 : 0) | (p->out_dtype == GDN_BF16 ? F_OUT_BF16 : 0) |

@@ -281,6 +281,7 @@ struct Unit {
   int tok0, tok1;    // token range
   int status;
   int err;
+  int64_t p0, L;     // paged suffix: first CSR position and tokens of the sequence
 };
 
 __device__ __forceinline__ int64_t ld_index(const void* base, int64_t i, bool i64) {
@@ -310,11 +311,45 @@ __device__ __forceinline__ void resolve_page_rows(const void* indices, const voi
   write = w;
 }
 
+// The last T tokens of a paged sequence: a page holds the state after its
+// last token, so with L = (pages - 1) * page_size + last_page_len the state
+// is read from the page of position L-T-1 and the final state goes to the
+// last page (pages filled inside the suffix are written by the kernel's
+// token loop, see suffix_snapshot_page).
+__device__ __forceinline__ void resolve_suffix(const StepParams& p, int b, Unit& u) {
+  const bool i64 = (p.flags & F_IDX64) != 0;
+  u.src = u.dst = -1;
+  const int64_t p0 = ld_index(p.indptr, b, i64);
+  const int64_t p1 = ld_index(p.indptr, b + 1, i64);
+  const int64_t len = ld_index(p.lastlen, b, i64);
+  if (p0 < 0 || p1 > p.nnz) { u.err |= E_PAGE_RANGE; return; }
+  if (p1 <= p0 || len < 1 || len > p.page_size) { u.err |= E_PAGE_TABLE; return; }
+  const int64_t L = (p1 - p0 - 1) * p.page_size + len;
+  if (L < p.T + 1) { u.err |= E_PAGE_TABLE; return; }
+  const int64_t r = ld_index(p.idx, p0 + (L - p.T - 1) / p.page_size, i64);
+  const int64_t w = ld_index(p.idx, p1 - 1, i64);
+  if (r < 0 || r >= p.num_slots || w < 0 || w >= p.num_slots) { u.err |= E_PAGE_RANGE; return; }
+  u.src = r;
+  u.dst = w;
+  u.p0 = p0;
+  u.L = L;
+}
+
+// Page that receives the state after suffix token t (not the last one), or
+// -1: the page whose last position is L-T+t, when that position closes a page.
+__device__ __forceinline__ int64_t suffix_snapshot_page(const StepParams& p, const Unit& u, int t) {
+  const int64_t pos = u.L - p.T + t;
+  if (t >= p.T - 1 || (pos % p.page_size) != p.page_size - 1) return -1;
+  return ld_index(p.idx, u.p0 + pos / p.page_size, (p.flags & F_IDX64) != 0);
+}
+
 template <int IDX>
 __device__ __forceinline__ Unit resolve_unit(const StepParams& p, int b) {
   Unit u;
   u.status = U_OK;
   u.err = 0;
+  u.p0 = 0;
+  u.L = 0;
   const bool i64 = (p.flags & F_IDX64) != 0;
   if constexpr (IDX == IDX_SLOTS) {
     if (p.flags & F_VARLEN) {
@@ -334,6 +369,12 @@ __device__ __forceinline__ Unit resolve_unit(const StepParams& p, int b) {
     u.src = u.dst = s;
     if (s < 0) u.status = U_PAD;
     else if (s >= p.num_slots) { u.status = U_PAD; u.err |= E_SLOT_RANGE; }
+  } else if (p.T > 1) {
+    // suffix of T tokens (see resolve_suffix)
+    u.tok0 = b * p.T;
+    u.tok1 = u.tok0 + p.T;
+    resolve_suffix(p, b, u);
+    if (u.err) u.status = U_PAD;
   } else {
     u.tok0 = b;
     u.tok1 = b + 1;

@@ -167,6 +167,24 @@ step_seq(const StepParams p) {
   [[maybe_unused]] float s_last = 0.0f;
   [[maybe_unused]] uint32_t codes[NR][EPL / 4];
 
+  // store the tile (in its storage format) to pool slot/page `slot`
+  auto store_tile = [&](int64_t slot) {
+    char* dst = reinterpret_cast<char*>(p.pool) + (slot * p.HV + hv) * head_bytes;
+    if constexpr (SDT == ST_FP8) {
+#pragma unroll
+      for (int jj = 0; jj < NR; ++jj) {
+        char* a = dst + vec_off(jj);
+        if constexpr (EPL == 16) st_stream16(a, make_uint4(codes[jj][0], codes[jj][1], codes[jj][2], codes[jj][3]));
+        else if constexpr (EPL == 8) __stcs(reinterpret_cast<uint2*>(a), make_uint2(codes[jj][0], codes[jj][1]));
+        else __stcs(reinterpret_cast<unsigned int*>(a), codes[jj][0]);
+      }
+      if (threadIdx.x == 0) p.scales[(slot * p.HV + hv) * n_scale + stile] = s_last;
+    } else {
+#pragma unroll
+      for (int jj = 0; jj < NR; ++jj) SV::store(dst + vec_off(jj) * ST::BYTES, SV::encode(S[jj]));
+    }
+  };
+
   for (int t0 = u.tok0; t0 < u.tok1; t0 += TC) {
     const int nt = min(TC, u.tok1 - t0);
     // ---- prologue of the chunk: one warp per token
@@ -412,25 +430,23 @@ step_seq(const StepParams p) {
         }
       }
       if (writer) st_out1(p.out, ((int64_t)tok * p.HV + hv) * V + out_col, o_mine, out_bf16);
+      if constexpr (IDX == IDX_PAGED) {
+        // a page that fills inside a multi-token suffix keeps this state
+        if (p.T > 1) {
+          const int64_t page = suffix_snapshot_page(p, u, tok - u.tok0);
+          if (page >= p.num_slots) {
+            if (threadIdx.x == 0) raise_err(p.err, E_PAGE_RANGE);
+          } else if (page >= 0) {
+            store_tile(page);
+          }
+        }
+      }
     }
     __syncthreads();  // the next chunk's prologue overwrites the token buffers
   }
 
   // ---- store the state once, after the last token
-  char* dst = reinterpret_cast<char*>(p.pool) + (u.dst * p.HV + hv) * head_bytes;
-  if constexpr (SDT == ST_FP8) {
-#pragma unroll
-    for (int jj = 0; jj < NR; ++jj) {
-      char* a = dst + vec_off(jj);
-      if constexpr (EPL == 16) st_stream16(a, make_uint4(codes[jj][0], codes[jj][1], codes[jj][2], codes[jj][3]));
-      else if constexpr (EPL == 8) __stcs(reinterpret_cast<uint2*>(a), make_uint2(codes[jj][0], codes[jj][1]));
-      else __stcs(reinterpret_cast<unsigned int*>(a), codes[jj][0]);
-    }
-    if (threadIdx.x == 0) p.scales[(u.dst * p.HV + hv) * n_scale + stile] = s_last;
-  } else {
-#pragma unroll
-    for (int jj = 0; jj < NR; ++jj) SV::store(const_cast<char*>(dst) + vec_off(jj) * ST::BYTES, SV::encode(S[jj]));
-  }
+  store_tile(u.dst);
 }
 
 }  // namespace gdn

@@ -152,23 +152,32 @@ typedef struct gdn_decode_slots_params {
 
 int gdn_decode_slots(const gdn_decode_slots_params* p, gdn_stream_t stream);
 
-/* GDN single-token decode on a paged pool (num_slots = num_pages).
- *  q, k [B, 1, H, K]; v [B, 1, HV, V]; a, b [B, 1, HV]; A_log, dt_bias [HV];
+/* GDN decode of the last T tokens of every sequence on a paged pool
+ * (num_slots = num_pages); a page holds the state after its last token.
+ *  q, k [B, T, H, K]; v [B, T, HV, V]; a, b [B, T, HV]; A_log, dt_bias [HV];
  *  page_indices [nnz], page_indptr [B+1], last_page_len [B] (index_dtype):
- *    CSR page table; the decoded token is the last token of its sequence and
- *    last_page_len counts it (in [1, page_size]).
+ *    CSR page table; the decoded tokens are the last T tokens of their
+ *    sequence and last_page_len counts the tokens of the last page,
+ *    including them (in [1, page_size]).
+ *  out [B, T, HV, V].
+ * T == 1, copy-on-new-page: when last_page_len[b] == 1 the state is read
+ * from the page before the last and written to the last page, so the
+ * previous page (possibly shared) is not modified; otherwise the last page
+ * is updated in place. A sequence that opens a page must own at least two
+ * pages. page_size <= 0 disables the last_page_len upper-bound check.
  *  slots: optional [B, 2] int64 rows (read_page, write_page) as written by
  *    gdn_paged_decode_slots for the same table; used as given, not checked
  *    against the table. NULL: the kernel resolves the rows itself in its
  *    prologue (no extra launch).
- * Copy-on-new-page: when last_page_len[b] == 1 the state is read from the
- * page before the last and written to the last page, so the previous page
- * (possibly shared) is not modified; otherwise the last page is updated in
- * place. A sequence that opens a page must own at least two pages.
- * page_size <= 0 disables the last_page_len upper-bound check. */
+ * T > 1 (a short suffix; page_size required, slots must be NULL): with
+ * L = (pages - 1) * page_size + last_page_len tokens, the suffix is
+ * positions L-T .. L-1 and at least one token must precede it. The state
+ * is read from the page of position L-T-1; every page whose last position
+ * falls inside the suffix receives the state after that position; the final
+ * state goes to the last page. Pages before the read page are untouched. */
 typedef struct gdn_decode_paged_params {
   int32_t struct_size; /* sizeof(gdn_decode_paged_params) */
-  int32_t B, H, HV, K, V;
+  int32_t B, T, H, HV, K, V;
   int32_t in_dtype, out_dtype, index_dtype, readout, use_qk_l2norm;
   int32_t page_size;
   float scale;

@@ -215,30 +215,35 @@ def store_state(payload, layout, state_dtype):
 # one (sequence, value head) over its tokens
 # ----------------------------------------------------------------------------
 
-def run_unit(S0, tokens, state_dtype, readout_mode="working", block_v=64):
-    """Run one state over its tokens.
+def step_unit(S0, tokens, state_dtype, readout_mode="working", block_v=64):
+    """Run one state over its tokens, yielding (o, payload) after every token.
 
     ``S0``: float64 [K, V] (already decoded). ``tokens``: iterable of
-    ``(q_hat, k_hat, v, alpha, beta)``. Returns (outputs [T, V], final payload
-    or None when there are no tokens).
-
-    fp32 states carry float64 between tokens and are rounded once when
-    stored; bf16 and fp8 states pass through their storage after every token.
+    ``(q_hat, k_hat, v, alpha, beta)``. ``payload`` is what the pool would
+    hold if the state were stored right then. fp32 states carry float64
+    between tokens (a stored copy is rounded once); bf16 and fp8 states pass
+    through their storage after every token (a write event).
     """
     S = S0
-    outs = []
-    payload = None
     for (q_hat, k_hat, v, alpha, beta) in tokens:
         o, S = gated_delta_step(S, q_hat, k_hat, v, alpha, beta)
-        if state_dtype != "f32":
+        if state_dtype == "f32":
+            _, payload = write_event(S, "f32")
+        else:
             S, payload = write_event(S, state_dtype, block_v)
             if readout_mode == "stored":
                 o = readout(S, q_hat)
+        yield o, payload
+
+
+def run_unit(S0, tokens, state_dtype, readout_mode="working", block_v=64):
+    """All of a unit's tokens: (outputs [T, V], final payload or None when
+    there are no tokens)."""
+    outs, payload = [], None
+    for o, payload in step_unit(S0, tokens, state_dtype, readout_mode, block_v):
         outs.append(o)
     if not outs:
         return np.zeros((0, S0.shape[1])), None
-    if state_dtype == "f32":
-        _, payload = write_event(S, "f32")
     return np.stack(outs), payload
 
 
@@ -320,41 +325,78 @@ def resolve_pages(page_indices, page_indptr, last_page_len, bb):
     return read, write
 
 
+def suffix_pages(page_indices, page_indptr, last_page_len, page_size, T, bb):
+    """Pages a T-token suffix of sequence bb touches.
+
+    The sequence holds L = (pages - 1) * page_size + last_page_len tokens;
+    the suffix is its last T tokens (positions L-T .. L-1) and at least one
+    token precedes it. A page holds the state after its last token, so the
+    state is read from the page of position L-T-1, every page whose last
+    position falls inside the suffix (except the last page) receives the
+    state after that position, and the final state goes to the last page.
+    For T == 1 this is the copy-on-new-page rule.
+    Returns (read_page, [(t, page)], last_page) with t the suffix index
+    after which the snapshot is taken.
+    """
+    p0, p1 = int(page_indptr[bb]), int(page_indptr[bb + 1])
+    npg = p1 - p0
+    L = (npg - 1) * page_size + int(last_page_len[bb])
+    if npg < 1 or L < T + 1:
+        raise ValueError("a suffix needs at least one token before it")
+    read = int(page_indices[p0 + (L - T - 1) // page_size])
+    snaps = [(t, int(page_indices[p0 + (L - T + t) // page_size])) for t in range(T - 1)
+             if (L - T + t) % page_size == page_size - 1]
+    return read, snaps, int(page_indices[p1 - 1])
+
+
 def gdn_decode_paged(q, k, v, a, b, A_log, dt_bias, state_pool, page_indices, page_indptr,
                      last_page_len, *, state_dtype="f32", state_scales=None, block_v=64,
                      scale=None, use_qk_l2norm=True, readout_mode="working", slots=None,
-                     units=None):
-    """Single-token GDN decode on a paged pool stored ``[num_pages, HV, V, K]``.
+                     units=None, page_size=None, layout="V_FIRST"):
+    """GDN decode of the last T tokens of each sequence on a paged pool
+    (stored ``[num_pages, HV, V, K]`` for V_FIRST).
 
-    q, k: [B, 1, H, K]; v: [B, 1, HV, V]; a, b: [B, 1, HV]. ``slots``, when
-    given, is a [B, 2] array of (read_page, write_page) used as is (the page
-    says precomputed rows are not checked against the page table).
-    Returns (out [B, 1, HV, V], writes keyed by (write_page, hv)).
+    q, k: [B, T, H, K]; v: [B, T, HV, V]; a, b: [B, T, HV]. T == 1 follows
+    the copy-on-new-page rule and needs no page_size; ``slots``, when given
+    for T == 1, is a [B, 2] array of (read_page, write_page) used as is (the
+    page says precomputed rows are not checked against the page table).
+    T > 1 needs page_size and writes a snapshot to every page that fills up
+    inside the suffix (``suffix_pages``).
+    Returns (out [B, T, HV, V], writes keyed by (page, hv)).
     """
     q = np.asarray(q, np.float64); k = np.asarray(k, np.float64)
     v = np.asarray(v, np.float64); a = np.asarray(a, np.float64); b = np.asarray(b, np.float64)
     B, T, H, K = q.shape
-    if T != 1:
-        raise ValueError("paged decode takes exactly one token per sequence")
     HV, V = v.shape[2], v.shape[3]
+    if T > 1 and not page_size:
+        raise ValueError("a multi-token suffix needs page_size")
     sc = _scale_of(scale, K)
-    out = np.full((B, 1, HV, V), np.nan) if units is not None else np.zeros((B, 1, HV, V))
+    out = np.full((B, T, HV, V), np.nan) if units is not None else np.zeros((B, T, HV, V))
     writes = {}
     todo = [(bb, hv) for bb in range(B) for hv in range(HV)] if units is None else list(units)
     for (bb, hv) in todo:
-        if slots is not None:
-            read, write = int(slots[bb][0]), int(slots[bb][1])
+        if T == 1:
+            if slots is not None:
+                read, write = int(slots[bb][0]), int(slots[bb][1])
+            else:
+                read, write = resolve_pages(page_indices, page_indptr, last_page_len, bb)
+            snaps = []
         else:
-            read, write = resolve_pages(page_indices, page_indptr, last_page_len, bb)
+            read, snaps, write = suffix_pages(page_indices, page_indptr, last_page_len, page_size, T, bb)
         h = key_head_of(hv, H, HV)
-        S0 = load_state(state_pool[read, hv], "V_FIRST", state_dtype,
+        S0 = load_state(state_pool[read, hv], layout, state_dtype,
                         None if state_scales is None else state_scales[read, hv], block_v)
-        qh, kh = prepare_qk(q[bb, 0, h], k[bb, 0, h], sc, use_qk_l2norm)
-        tok = (qh, kh, v[bb, 0, hv], gdn_alpha(A_log[hv], a[bb, 0, hv], dt_bias[hv]),
-               beta_of(b[bb, 0, hv]))
-        o, payload = run_unit(S0, [tok], state_dtype, readout_mode, block_v)
-        out[bb, :, hv, :] = o
-        writes[(write, hv)] = store_state(payload, "V_FIRST", state_dtype)
+        toks = []
+        for t in range(T):
+            qh, kh = prepare_qk(q[bb, t, h], k[bb, t, h], sc, use_qk_l2norm)
+            toks.append((qh, kh, v[bb, t, hv], gdn_alpha(A_log[hv], a[bb, t, hv], dt_bias[hv]),
+                         beta_of(b[bb, t, hv])))
+        snap_at = dict(snaps)
+        for t, (o, payload) in enumerate(step_unit(S0, toks, state_dtype, readout_mode, block_v)):
+            out[bb, t, hv, :] = o
+            if t in snap_at:
+                writes[(snap_at[t], hv)] = store_state(payload, layout, state_dtype)
+        writes[(write, hv)] = store_state(payload, layout, state_dtype)
     return out, writes
 
 

@@ -198,12 +198,17 @@ def gdn_slots_case(seed, B, T, H, HV, K, V, num_slots, layout="V_FIRST", state_d
 
 def gdn_paged_case(seed, B, H, HV, K, V, page_size, max_len, n_share, share_pages, force_lens=None,
                    state_dtype="f32", in_dtype="bf16", out_dtype="f32", index_dtype="i32",
-                   use_slots=False, units=None, spare_pages=0, readout="working", layout="V_FIRST"):
+                   use_slots=False, units=None, spare_pages=0, readout="working", layout="V_FIRST", T=1,
+                   min_len=2):
     pt = W.paged_table(seed, B, page_size, max_len, n_share, share_pages, force_lens,
-                       spare_pages).cast(index_dtype)
-    t = W.gdn_tokens(seed, B, 1, H, HV, K, V, in_dtype)
-    rows = O.paged_decode_slots(pt.page_indices, pt.page_indptr, pt.last_page_len)
-    touched = sorted(set(rows.reshape(-1).tolist()))
+                       spare_pages, min_len=max(min_len, T + 1)).cast(index_dtype)
+    t = W.gdn_tokens(seed, B, T, H, HV, K, V, in_dtype)
+    rows = O.paged_decode_slots(pt.page_indices, pt.page_indptr, pt.last_page_len) if T == 1 else None
+    if T == 1:
+        touched = sorted(set(rows.reshape(-1).tolist()))
+    else:
+        touched = sorted({pg for bb in range(B)
+                          for pg in ([O.suffix_pages(pt.page_indices, pt.page_indptr, pt.last_page_len, page_size, T, bb)[0]])})
     pool, scales = W.device_pool(seed, pt.num_pages, HV, K, V, layout, state_dtype,
                                  exact_slots=touched)
     snap = pool.clone()
@@ -230,17 +235,17 @@ def gdn_paged_case(seed, B, H, HV, K, V, page_size, max_len, n_share, share_page
     ref_out, writes = O.gdn_decode_paged(
         t["q"], t["k"], t["v"], t["a"], t["b"], t["A_log"], t["dt_bias"], states, pt.page_indices,
         pt.page_indptr, pt.last_page_len, state_dtype=state_dtype, state_scales=sc,
-        readout_mode=readout, units=todo)
+        readout_mode=readout, units=todo, page_size=page_size, layout=layout)
     out_h = host(out)
-    res["out_err"] = check_outputs(out_h, ref_out, todo, lambda x, b, hv: x[b, 0, hv, :],
+    res["out_err"] = check_outputs(out_h, ref_out, todo, lambda x, b, hv: x[b, :, hv, :],
                                    TOL[state_dtype], out_dtype)
     # written pages: compare the sampled units; every other page must be bit-identical
-    write_pages = sorted(set(rows[:, 1].tolist()))
+    write_pages = sorted({pg for (pg, _) in writes}) if units is None else sorted(set(rows[:, 1].tolist()))
     wp = torch.tensor(write_pages, device="cuda")
     after_w = pool_host(pool[wp])
     sc_after_w = scales[wp].cpu().numpy() if scales is not None else None
-    pos = {p: i for i, p in enumerate(write_pages)}
-    sub_writes = {(pos[p], hv): w for (p, hv), w in writes.items()}
+    pos = {pg: i for i, pg in enumerate(write_pages)}
+    sub_writes = {(pos[pg], hv): w for (pg, hv), w in writes.items()}
     res["state_err"] = check_state(after_w, sc_after_w, sub_writes, state_dtype, layout)
     keep = torch.ones(pt.num_pages, dtype=torch.bool, device="cuda")
     keep[wp] = False
@@ -248,6 +253,7 @@ def gdn_paged_case(seed, B, H, HV, K, V, page_size, max_len, n_share, share_page
     if scales is not None:
         assert torch.equal(scales[keep], sc_snap[keep])
     res["write_pages"] = write_pages
+    res["writes"] = writes
     return res
 
 

@@ -459,4 +459,70 @@ def pin_fp8_state_codec_per_tile():
         assert s == scales[j] and np.array_equal(c, codes[:, 4 * j:4 * j + 4])
 
 
+
+
+# ----------------------------------------------------------------------------
+# multi-token suffix on a paged pool
+# ----------------------------------------------------------------------------
+
+def read_suffix_cases():
+    cases = []
+    with open(os.path.join(GOLDEN, "paged_suffix_cases.txt")) as f:
+        for line in f:
+            line = line.split("#")[0].strip()
+            if not line:
+                continue
+            ind, ptr, last, ps, T, read, snaps, final = [p.strip() for p in line.split(";")]
+            snap = [] if snaps == "-" else [tuple(int(y) for y in z.split(":")) for z in snaps.split()]
+            cases.append(([int(x) for x in ind.split()], [int(x) for x in ptr.split()], [int(last)],
+                          int(ps), int(T), int(read), snap, int(final)))
+    return cases
+
+
+def pin_paged_suffix_rule():
+    """The suffix page rule on hand-derived tables, and T == 1 agrees with
+    the copy-on-new-page rule on every table of the single-token fixture."""
+    for ind, ptr, last, ps, T, read, snaps, final in read_suffix_cases():
+        got = O.suffix_pages(ind, ptr, last, ps, T, 0)
+        assert got == (read, snaps, final), (ind, ptr, last, ps, T, got)
+    for ind, ptr, last, exp in read_paged_cases():
+        for bb in range(len(ptr) - 1):
+            n = ptr[bb + 1] - ptr[bb]
+            ps = 64
+            if last[bb] > ps:
+                continue
+            r, snaps, w = O.suffix_pages(ind, ptr, last, ps, 1, bb)
+            assert (r, w) == exp[bb] and snaps == []
+
+
+def pin_paged_suffix_equals_single_steps():
+    """A T-token suffix equals T single-token paged calls on the sequence
+    growing by one token each time, threaded through the pool."""
+    ps, HV, K, V, H = 3, 2, 4, 4, 1
+    ind = [4, 0, 2, 5, 1]
+    L, T = 14, 7                       # 5 pages: positions 0..14? L = 4*3 + 2
+    last = [L - ps * (len(ind) - 1)]
+    pool = _tiny_pool(81, 6, HV, K, V).astype(np.float64)
+    t = _tiny_tokens(82, 1, T, H, HV, K, V)
+    out, writes = O.gdn_decode_paged(t["q"], t["k"], t["v"], t["a"], t["b"], t["A_log"], t["dt_bias"], pool,
+                                     ind, [0, len(ind)], last, page_size=ps)
+    p = pool.copy()
+    for s in range(T):
+        Ls = L - T + s + 1
+        npg = -(-Ls // ps)
+        o1, w1 = O.gdn_decode_paged(t["q"][:, s:s + 1], t["k"][:, s:s + 1], t["v"][:, s:s + 1], t["a"][:, s:s + 1],
+                                    t["b"][:, s:s + 1], t["A_log"], t["dt_bias"], p, ind[:npg], [0, npg],
+                                    [Ls - ps * (npg - 1)])
+        assert np.allclose(o1[0, 0], out[0, s], rtol=0, atol=1e-6)
+        for (page, hv), (st, _) in w1.items():
+            p[page, hv] = st
+    for (page, hv), (st, _) in writes.items():
+        assert np.allclose(p[page, hv], st, rtol=0, atol=1e-6), (page, hv)
+    # pages the suffix does not reach keep their content
+    touched = {pg for (pg, _) in writes}
+    for pg in range(6):
+        if pg not in touched:
+            assert np.array_equal(p[pg], pool[pg])
+
+
 ALL_PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]

@@ -121,7 +121,7 @@ def test_null_params_and_status_strings(lib):
 def test_paged_validation(lib):
     p = G.gdn_decode_paged_params()
     p.struct_size = ctypes.sizeof(p)
-    p.B, p.H, p.HV, p.K, p.V, p.nnz = 2, 1, 2, 128, 128, 4
+    p.B, p.T, p.H, p.HV, p.K, p.V, p.nnz = 2, 1, 1, 2, 128, 128, 4
     for f in ("q", "k", "v", "a", "b", "A_log", "dt_bias", "out"):
         setattr(p, f, FAKE)
     p.pool = G.gdn_state_pool(FAKE, None, 4, G.GDN_F32, G.GDN_V_FIRST, 64, 0)
@@ -130,6 +130,10 @@ def test_paged_validation(lib):
     assert lib.gdn_decode_paged(ctypes.byref(p), None) == G.GDN_ERR_INVALID_ARG
     p.nnz, p.B = 4, 0
     assert lib.gdn_decode_paged(ctypes.byref(p), None) == G.GDN_OK
+    p.B, p.T, p.page_size = 2, 3, 0          # a suffix needs page_size
+    assert lib.gdn_decode_paged(ctypes.byref(p), None) == G.GDN_ERR_INVALID_ARG
+    p.page_size, p.slots = 16, FAKE          # precomputed rows are single-token only
+    assert lib.gdn_decode_paged(ctypes.byref(p), None) == G.GDN_ERR_INVALID_ARG
 
 
 def test_kda_validation(lib):

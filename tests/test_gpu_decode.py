@@ -205,6 +205,30 @@ def test_paged_state_dtypes(state_dtype):
                    force_lens={0: 17}, state_dtype=state_dtype)
 
 
+@pytest.mark.parametrize("T,page_size", [(2, 16), (5, 4), (19, 4), (9, 8)])
+@pytest.mark.parametrize("state_dtype", ["f32", "bf16"])
+def test_paged_suffix(T, page_size, state_dtype):
+    """The last T tokens on a paged pool: read from the page of the token
+    before the suffix, a snapshot in every page that fills inside it, the
+    final state in the last page, every other page untouched."""
+    # suffixes start past the 2 shared pages, so no two sequences write one page
+    r = gdn_paged_case(34 + T, B=7, H=1, HV=2, K=128, V=128, page_size=page_size, max_len=60,
+                       n_share=2, share_pages=2, state_dtype=state_dtype, T=T,
+                       min_len=T + 2 * page_size + 1)
+    assert r["err"] == 0
+    n_snap = len(r["write_pages"]) - 7
+    if T - 1 >= page_size:   # a page boundary falls inside every suffix
+        assert n_snap >= 7
+
+
+@pytest.mark.parametrize("layout", ["V_FIRST", "K_FIRST"])
+def test_paged_suffix_layouts_and_fp8(layout):
+    gdn_paged_case(36, B=4, H=2, HV=4, K=128, V=128, page_size=8, max_len=40, n_share=0, share_pages=0,
+                   state_dtype="fp8_e4m3", T=6, layout=layout)
+    gdn_paged_case(37, B=4, H=2, HV=4, K=64, V=64, page_size=8, max_len=40, n_share=0, share_pages=0,
+                   T=3, layout=layout)
+
+
 def test_paged_full_size():
     w = W.WORKLOADS["paged"]
     r = gdn_paged_case(w.seed, w.B, w.H, w.HV, w.K, w.V, w.page_size, w.max_len, w.n_share, w.share_pages,

@@ -38,6 +38,15 @@ def _resolve_writing_old_page(page_indices, page_indptr, last_page_len, bb):
 
 
 _ORIG_RESOLVE = O.resolve_pages
+_ORIG_SUFFIX = O.suffix_pages
+
+
+def _suffix_read_too_late(page_indices, page_indptr, last_page_len, page_size, T, bb):
+    """Reads the page of position L-T (the suffix's first token) instead of L-T-1."""
+    read, snaps, final = _ORIG_SUFFIX(page_indices, page_indptr, last_page_len, page_size, T, bb)
+    p0, p1 = int(page_indptr[bb]), int(page_indptr[bb + 1])
+    L = (p1 - p0 - 1) * page_size + int(last_page_len[bb])
+    return int(page_indices[p0 + (L - T) // page_size]), snaps, final
 _ORIG_QUANT_TILE = formats.quantize_tile
 
 
@@ -81,6 +90,7 @@ MUTATIONS = {
                          if use else (np.asarray(q, float), np.asarray(k, float))),
     "new_page_ignored": (O, "resolve_pages", _resolve_ignoring_new_page),
     "write_to_read_page": (O, "resolve_pages", _resolve_writing_old_page),
+    "suffix_read_too_late": (O, "suffix_pages", _suffix_read_too_late),
     "bf16_truncates": (formats, "f32_to_bf16_bits",
                        lambda x: (np.ascontiguousarray(np.asarray(x, np.float32)).view(np.uint32) >> 16).astype(np.uint16)),
     "e4m3_half_away": (formats, "e4m3_encode", _e4m3_half_away),

@@ -176,8 +176,8 @@ class PageTable:
 
 
 def paged_table(seed, B, page_size, max_len, n_share, share_pages, force_lens=None,
-                spare_pages=0) -> PageTable:
-    """CSR page table of B sequences with lengths U[2, max_len].
+                spare_pages=0, min_len=2) -> PageTable:
+    """CSR page table of B sequences with lengths U[min_len, max_len].
 
     Sequences 0..n_share-1 share their first ``share_pages`` full pages and
     have lengths above the shared prefix (resampled), so that their last
@@ -188,10 +188,10 @@ def paged_table(seed, B, page_size, max_len, n_share, share_pages, force_lens=No
     """
     r = _rng(seed, _LENGTHS)
     prefix = share_pages * page_size
-    lens = r.integers(2, max_len + 1, size=B)
+    lens = r.integers(min_len, max_len + 1, size=B)
     for bb in range(min(n_share, B)):
         while lens[bb] <= prefix:
-            lens[bb] = r.integers(2, max_len + 1)
+            lens[bb] = r.integers(min_len, max_len + 1)
     for bb, L in (force_lens or {}).items():
         lens[bb] = L
     npages = -(-lens // page_size)
