@@ -33,7 +33,7 @@ bool ptrs_ok(std::initializer_list<const void*> vec16, std::initializer_list<std
     if (x.first == nullptr || !aligned(x.first, x.second)) return false;
   return true;
 }
-bool head_dim_ok(int x) { return x == 32 || x == 64 || x == 128; }
+bool head_dim_ok(int x) { return x == 32 || x == 64 || x == 128 || x == 256; }
 bool io_dtype_ok(int d) { return d == GDN_F32 || d == GDN_BF16; }
 bool state_dtype_ok(int d) { return d == GDN_F32 || d == GDN_BF16 || d == GDN_FP8_E4M3; }
 bool layout_ok(int l) { return l == GDN_K_FIRST || l == GDN_V_FIRST; }
@@ -102,11 +102,17 @@ int launch_one(StepParams p, int B, cudaStream_t s) {
   if constexpr (L == L_VFIRST && GATE == GATE_SCALAR) {
     if (p.T == 1) return launch_tile1<SDT, K, IDX>(p, B, s);
   }
-  if constexpr (L == L_KFIRST && SDT != ST_FP8) {
-    // 16 columns per warp: 4 warps when V allows a 64-column tile
-    if (p.V % 64 != 0) return launch_seq_nw<L, SDT, K, GATE, IDX, 2>(p, B, s);
+  if constexpr (L == L_KFIRST) {
+    constexpr int VTW = (K == 256) ? 8 : 16;  // columns per warp
+    if constexpr (SDT == ST_FP8) {
+      return launch_seq_nw<L, SDT, K, GATE, IDX, 64 / VTW>(p, B, s);  // the 64-column scale tile
+    } else {
+      if (p.V % (4 * VTW) != 0) return launch_seq_nw<L, SDT, K, GATE, IDX, 2>(p, B, s);
+      return launch_seq_nw<L, SDT, K, GATE, IDX, 4>(p, B, s);
+    }
+  } else {
+    return launch_seq_nw<L, SDT, K, GATE, IDX, (SDT == ST_FP8 && K == 256) ? 8 : 4>(p, B, s);
   }
-  return launch_seq_nw<L, SDT, K, GATE, IDX, 4>(p, B, s);
 }
 
 template <int L, int SDT, int GATE, int IDX>
@@ -115,6 +121,7 @@ int launch_k(const StepParams& p, int K, int B, cudaStream_t s) {
     case 32: return launch_one<L, SDT, 32, GATE, IDX>(p, B, s);
     case 64: return launch_one<L, SDT, 64, GATE, IDX>(p, B, s);
     case 128: return launch_one<L, SDT, 128, GATE, IDX>(p, B, s);
+    case 256: return launch_one<L, SDT, 256, GATE, IDX>(p, B, s);
     default: return GDN_ERR_INVALID_ARG;
   }
 }
@@ -158,8 +165,9 @@ __global__ void paged_rows_kernel(const void* indices, const void* indptr, const
 // One CTA per [K, 64] tile of one state. Thread t owns 16-element chunks
 // t, t + NT, ...; a chunk is 16 consecutive elements of one stored row.
 template <int K, int LAYOUT>
-__global__ void __launch_bounds__(128) fp8_quantize_kernel(const float* src, uint8_t* codes, float* scales, int V) {
-  constexpr int NT = 128, BV = 64, CHUNKS = K * BV / 16, PER = CHUNKS / NT;
+__global__ void __launch_bounds__(K == 256 ? 256 : 128) fp8_quantize_kernel(const float* src, uint8_t* codes,
+                                                                            float* scales, int V) {
+  constexpr int NT = (K == 256) ? 256 : 128, BV = 64, CHUNKS = K * BV / 16, PER = CHUNKS / NT;
   static_assert(CHUNKS % NT == 0, "tile must split over the CTA");
   __shared__ float s_amax[NT / 32];
   const int n_tiles = V / BV;
@@ -235,6 +243,7 @@ int launch_quantize(const float* src, uint8_t* codes, float* scales, int64_t n, 
     case 32: fp8_quantize_kernel<32, LAYOUT><<<g, 128, 0, s>>>(src, codes, scales, V); break;
     case 64: fp8_quantize_kernel<64, LAYOUT><<<g, 128, 0, s>>>(src, codes, scales, V); break;
     case 128: fp8_quantize_kernel<128, LAYOUT><<<g, 128, 0, s>>>(src, codes, scales, V); break;
+    case 256: fp8_quantize_kernel<256, LAYOUT><<<g, 256, 0, s>>>(src, codes, scales, V); break;
     default: return GDN_ERR_INVALID_ARG;
   }
   return launch_status();

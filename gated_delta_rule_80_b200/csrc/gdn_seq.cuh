@@ -52,9 +52,13 @@ struct ReduceScatterS {
 template <int SDT, int LAYOUT, int K, int NW>
 struct SeqShape {
   static constexpr int TC = 8;  // tokens per prologue chunk
-  // V_FIRST: 16-byte vectors; K_FIRST: 4 elements per lane, 16 columns per warp
-  static constexpr int EPL = (LAYOUT == L_VFIRST) ? 16 / StateTraits<SDT>::BYTES : 4;
-  static constexpr int VC = (LAYOUT == L_VFIRST) ? ((SDT == ST_FP8) ? 64 : 32) : 16 * NW;
+  // V_FIRST: 16-byte vectors (32 for a K=256 fp32 row, so that it fits a warp)
+  static constexpr int VB_V = (SDT == ST_F32 && K == 256) ? 32 : 16;
+  // K_FIRST: 4 elements per lane, CPL lanes per row segment (16 columns per
+  // warp; 8 for K = 256 so that a thread holds K/16 rows)
+  static constexpr int CPL = (K == 256) ? 2 : 4;
+  static constexpr int EPL = (LAYOUT == L_VFIRST) ? VB_V / StateTraits<SDT>::BYTES : 4;
+  static constexpr int VC = (LAYOUT == L_VFIRST) ? ((SDT == ST_FP8) ? 64 : (K == 256 ? 16 : 32)) : CPL * 4 * NW;
 };
 
 template <int SDT, int LAYOUT, int K, int GATE, int IDX, int NW>
@@ -66,16 +70,19 @@ step_seq(const StepParams p) {
   constexpr int EPL = SH::EPL;
   constexpr int VC = SH::VC;
   constexpr int VB = EPL * ST::BYTES;  // bytes per lane vector
-  static_assert(VB == 4 || VB == 8 || VB == 16, "vector width");
+  static_assert(VB == 4 || VB == 8 || VB == 16 || VB == 32, "vector width");
   constexpr bool VF = (LAYOUT == L_VFIRST);
+  constexpr int CPL = SH::CPL;        // K_FIRST lanes per row segment
+  constexpr int RG = 32 / CPL;        // K_FIRST row groups
   // V_FIRST geometry
-  constexpr int LPR = VF ? K / EPL : 4;
+  constexpr int LPR = VF ? K / EPL : CPL;
   constexpr int RPW = 32 / LPR;
-  constexpr int NR = VF ? VC / (NW * RPW) : K / 8;  // rows per thread
+  constexpr int NR = VF ? VC / (NW * RPW) : K / RG;  // rows per thread
   static_assert(!VF || (LPR >= 2 && LPR <= 32 && NR >= 1 && NR * NW * RPW == VC), "V_FIRST tile split");
-  static_assert(VF || (K % 8 == 0), "K_FIRST tile split");
+  static_assert(VF || (K % RG == 0 && VC == CPL * EPL * NW), "K_FIRST tile split");
   constexpr int NV = VF ? 2 * NR : 2 * EPL;  // partial sums per thread
   static_assert(!VF || NV <= LPR, "one finished sum per lane");
+  static_assert(VF || NV <= RG, "one finished sum per lane");
   constexpr int REP = VF ? LPR / NV : 1;
   constexpr int KPL = K / 32;
   constexpr int VPL = (VC + 31) / 32;
@@ -101,19 +108,20 @@ step_seq(const StepParams p) {
 
   // ---- thread geometry
   // V_FIRST: rows row0 + jj * RPW, elements kofs..kofs+EPL of each row.
-  // K_FIRST: rows g + 8 j, columns c0..c0+3 (all relative to the tile).
-  const int li = VF ? lane % LPR : lane % 4;
-  const int g = lane >> 2;  // K_FIRST row group
+  // K_FIRST: rows g + RG j, columns c0..c0+3 (all relative to the tile).
+  const int li = VF ? lane % LPR : lane % CPL;
+  const int g = lane / CPL;  // K_FIRST row group
   const int kofs = li * EPL;
   const int row0 = VF ? warp * NR * RPW + lane / LPR : 0;
-  const int c0 = VF ? 0 : warp * 16 + (lane & 3) * 4;
+  const int c0 = VF ? 0 : warp * CPL * 4 + li * 4;
   // the sum a lane finishes: V_FIRST value index li / REP (row, k or q);
-  // K_FIRST value index g (column g >> 1, k or q)
-  const int vidx = VF ? li / REP : g;
+  // K_FIRST value index from lane bits 4..2 (column >> 1, k or q); for
+  // CPL == 2, lane bit 1 is a replica
+  const int vidx = VF ? li / REP : (lane >> 2) & 7;
   const bool holds_q = (vidx & 1) != 0;
-  const int mycol = vidx >> 1;  // V_FIRST: row of the thread; K_FIRST: column of the quad
-  const int grp = VF ? lane - li : (lane & 3);
-  const bool writer = VF ? (!holds_q && (li % REP) == 0) : !holds_q;
+  const int mycol = vidx >> 1;  // V_FIRST: row of the thread; K_FIRST: column in the lane's 4
+  const int grp = VF ? lane - li : li;
+  const bool writer = VF ? (!holds_q && (li % REP) == 0) : (!holds_q && (CPL == 4 || (lane & 2) == 0));
 
   const Unit u = resolve_unit<IDX>(p, b);
   if (threadIdx.x == 0) raise_err(p.err, u.err);
@@ -127,16 +135,16 @@ step_seq(const StepParams p) {
   }
 
   // ---- state tile loads
-  using SV = StateVec<SDT, (VB == 16 ? 16 : 8)>;
+  using SV = StateVec<SDT, (VB >= 16 ? VB : 8)>;
   const int64_t head_bytes = (int64_t)K * V * ST::BYTES;
   const char* src = reinterpret_cast<const char*>(p.pool) + (u.src * p.HV + hv) * head_bytes;
   float S[NR][EPL];
   // element offset (within the head) of vector jj of this thread
   auto vec_off = [&](int jj) -> int64_t {
     if constexpr (VF) return (int64_t)(v0 + row0 + jj * RPW) * K + kofs;
-    else return (int64_t)(g + 8 * jj) * V + v0 + c0;
+    else return (int64_t)(g + RG * jj) * V + v0 + c0;
   };
-  if constexpr (VB == 16 || VB == 8) {
+  if constexpr (VB >= 8) {
     typename SV::T raw[NR];
 #pragma unroll
     for (int jj = 0; jj < NR; ++jj) raw[jj] = SV::load(src + vec_off(jj) * ST::BYTES);
@@ -271,7 +279,7 @@ step_seq(const StepParams p) {
         for (int c = 0; c < EPL / 2; ++c) { ak[c] = make_float2(0.f, 0.f); aq[c] = make_float2(0.f, 0.f); }
 #pragma unroll
         for (int jj = 0; jj < NR; ++jj) {
-          const int r = g + 8 * jj;
+          const int r = g + RG * jj;
           kw[jj] = s_k[tt][r];
           float wk = kw[jj], wq = s_q[tt][r];
           if constexpr (GATE == GATE_VECTOR) {
@@ -297,7 +305,7 @@ step_seq(const StepParams p) {
       }
       float mine;
       if constexpr (VF) mine = ReduceScatterS<NV, LPR / 2, 1>::run(x, lane);
-      else mine = ReduceScatterS<NV, 16, 4>::run(x, lane);
+      else mine = ReduceScatterS<NV, 16, CPL>::run(x, lane);
       constexpr int PAIR = VF ? REP : 4;  // lane offset between the k and q sums of one row/column
       const float other = __shfl_xor_sync(kFull, mine, PAIR);
       const float dk = holds_q ? other : mine;
@@ -318,7 +326,7 @@ step_seq(const StepParams p) {
         for (int jj = 0; jj < NR; ++jj) uu[jj] = __shfl_sync(kFull, u_mine, grp + 2 * jj * REP);
       } else {
 #pragma unroll
-        for (int c = 0; c < EPL; ++c) uu[c] = __shfl_sync(kFull, u_mine, (2 * c) * 4 + grp);
+        for (int c = 0; c < EPL; ++c) uu[c] = __shfl_sync(kFull, u_mine, (2 * c) * 4 + grp);  // lane bit 1 = 0
       }
       // S' = diag(alpha) S + k^ u^T
 #pragma unroll
@@ -336,7 +344,7 @@ step_seq(const StepParams p) {
             u2 = make_float2(uu[e], uu[e + 1]);
             if constexpr (GATE == GATE_SCALAR) f2 = make_float2(alpha, alpha);
             else {
-              const float a = s_a[tt][g + 8 * jj];
+              const float a = s_a[tt][g + RG * jj];
               f2 = make_float2(a, a);
             }
           }
@@ -416,7 +424,7 @@ step_seq(const StepParams p) {
             for (int c = 0; c < EPL; ++c) y[c] = 0.f;
 #pragma unroll
             for (int jj = 0; jj < NR; ++jj) {
-              const float qh = s_q[tt][g + 8 * jj];
+              const float qh = s_q[tt][g + RG * jj];
 #pragma unroll
               for (int c = 0; c < EPL; ++c) y[c] = fmaf(qh, S[jj][c], y[c]);
             }
@@ -425,7 +433,7 @@ step_seq(const StepParams p) {
               x[2 * c] = y[c];
               x[2 * c + 1] = 0.f;
             }
-            o_mine = ReduceScatterS<NV, 16, 4>::run(x, lane);
+            o_mine = ReduceScatterS<NV, 16, CPL>::run(x, lane);
           }
         }
       }

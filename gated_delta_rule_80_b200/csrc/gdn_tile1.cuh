@@ -26,13 +26,14 @@ namespace gdn {
 
 template <int SDT, int K>
 struct Tile1Shape {
-  static constexpr int VT = (SDT == ST_FP8) ? 64 : 32;   // fp8: the [K, 64] scale tile
-  static constexpr int NW = 4;
-  // bytes one lane moves per row
-  static constexpr int VB = 16;
+  // rows per tile: fp8 the [K, 64] scale tile; otherwise 16 KiB of fp32 state
+  static constexpr int VT = (SDT == ST_FP8) ? 64 : (K == 256 ? 16 : 32);
+  static constexpr int NW = (SDT == ST_FP8 && K == 256) ? 8 : 4;
+  // bytes one lane moves per row: a K=256 fp32 row needs 32 to fit a warp
+  static constexpr int VB = (SDT == ST_F32 && K == 256) ? 32 : 16;
   // resident CTAs per SM the register budget is sized for (fp8 holds 64
   // decoded elements per thread)
-  static constexpr int MIN_CTAS = (SDT == ST_FP8) ? 4 : 8;
+  static constexpr int MIN_CTAS = (SDT == ST_FP8) ? (NW == 8 ? 2 : 4) : 8;
 };
 
 // Vector of VB stored bytes: load/store and decode/encode.
@@ -45,6 +46,21 @@ template <int SDT> struct StateVec<SDT, 16> {
   __device__ __forceinline__ static void decode(T v, float* x) { decode16<SDT>(v, x); }
   __device__ __forceinline__ static T encode(const float* x) { return encode16<SDT>(x); }
   __device__ __forceinline__ static T zero() { return make_uint4(0u, 0u, 0u, 0u); }
+};
+template <int SDT> struct StateVec<SDT, 32> {
+  struct T { uint4 a, b; };
+  static constexpr int EPL = 2 * StateTraits<SDT>::EPL;
+  __device__ __forceinline__ static T load(const char* p) { return T{ld_stream16(p), ld_stream16(p + 16)}; }
+  __device__ __forceinline__ static void store(char* p, T v) {
+    st_stream16(p, v.a);
+    st_stream16(p + 16, v.b);
+  }
+  __device__ __forceinline__ static void decode(T v, float* x) {
+    decode16<SDT>(v.a, x);
+    decode16<SDT>(v.b, x + EPL / 2);
+  }
+  __device__ __forceinline__ static T encode(const float* x) { return T{encode16<SDT>(x), encode16<SDT>(x + EPL / 2)}; }
+  __device__ __forceinline__ static T zero() { return T{make_uint4(0u, 0u, 0u, 0u), make_uint4(0u, 0u, 0u, 0u)}; }
 };
 template <> struct StateVec<ST_BF16, 8> {
   using T = uint2;

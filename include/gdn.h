@@ -127,8 +127,8 @@ typedef struct gdn_state_pool {
  *  state_indices [B] (index_dtype): pool slot of each sequence; read and
  *                written in place after the last token.
  *  out      [B, T, HV, V]  out_dtype (F32 or BF16)
- * Constraints: HV % H == 0; K in {32, 64, 128}; V in {32, 64, 128}; fp8
- * state needs block_v == 64 and V % 64 == 0.
+ * Constraints: HV % H == 0; K and V in {32, 64, 128, 256}; fp8 state needs
+ * block_v == 64 and V % 64 == 0.
  * T > 1 runs the tokens of each sequence in order with the state held on
  * chip (a short suffix); bf16/fp8 states pass through their storage format
  * after every token. */

@@ -90,7 +90,8 @@ def _slots_params(**kw):
 @pytest.mark.parametrize("kw,expected", [
     (dict(struct_size=8), G.GDN_ERR_INVALID_ARG),
     (dict(K=48), G.GDN_ERR_INVALID_ARG),
-    (dict(V=256), G.GDN_ERR_INVALID_ARG),
+    (dict(V=512), G.GDN_ERR_INVALID_ARG),
+    (dict(K=96), G.GDN_ERR_INVALID_ARG),
     (dict(H=3), G.GDN_ERR_INVALID_ARG),
     (dict(B=-1), G.GDN_ERR_INVALID_ARG),
     (dict(in_dtype=2), G.GDN_ERR_INVALID_ARG),

@@ -371,7 +371,7 @@ def _adversarial_states(N, K, V, layout, seed=51):
 
 
 @pytest.mark.parametrize("layout", ["V_FIRST", "K_FIRST"])
-@pytest.mark.parametrize("K,V", [(128, 128), (32, 64), (64, 128)])
+@pytest.mark.parametrize("K,V", [(128, 128), (32, 64), (64, 128), (256, 256), (256, 64)])
 def test_fp8_codec_bit_exact(layout, K, V):
     N = 9
     x = _adversarial_states(N, K, V, layout)
@@ -395,3 +395,31 @@ def test_fp8_large_batch_full_size_sampled():
     units = sorted({(int(b), int(h)) for b, h in zip(r.integers(0, w.B, 400), r.integers(0, w.HV, 400))})
     gdn_slots_case(w.seed, w.B, w.T, w.H, w.HV, w.K, w.V, w.num_slots, state_dtype="fp8_e4m3",
                    in_dtype="bf16", out_dtype="bf16", units=units)
+
+
+# ----------------------------------------------------------------------------
+# head dims of 256
+# ----------------------------------------------------------------------------
+
+@pytest.mark.parametrize("layout", ["V_FIRST", "K_FIRST"])
+@pytest.mark.parametrize("state_dtype", ["f32", "bf16", "fp8_e4m3"])
+@pytest.mark.parametrize("T", [1, 3])
+def test_head_dim_256(layout, state_dtype, T):
+    gdn_slots_case(61 + T, B=3, T=T, H=1, HV=2, K=256, V=256, num_slots=5, layout=layout,
+                   state_dtype=state_dtype)
+
+
+@pytest.mark.parametrize("K,V", [(256, 64), (64, 256), (256, 32), (32, 256)])
+@pytest.mark.parametrize("layout", ["V_FIRST", "K_FIRST"])
+def test_head_dim_256_mixed(K, V, layout):
+    gdn_slots_case(63, B=2, T=2, H=1, HV=2, K=K, V=V, num_slots=3, layout=layout, in_dtype="f32")
+
+
+@pytest.mark.parametrize("layout", ["K_FIRST", "V_FIRST"])
+def test_kda_head_dim_256(layout):
+    kda_case(64, B=3, Hk=2, HV=2, K=256, V=256, num_slots=4, max_len=4, layout=layout)
+
+
+def test_paged_head_dim_256():
+    gdn_paged_case(65, B=5, H=1, HV=2, K=256, V=256, page_size=8, max_len=40, n_share=2, share_pages=1,
+                   force_lens={0: 9})
