@@ -10,6 +10,7 @@ Functions (same names as the C entry points):
 
 * ``gdn_decode_slots``      GDN decode of T >= 1 tokens on a slot pool
 * ``gdn_decode_paged``      GDN single-token decode on a paged pool
+* ``gdn_prefill_paged``     append varlen token runs to paged sequences
 * ``gdn_paged_decode_slots`` (read_page, write_page) rows for a page table
 * ``kda_decode_varlen``     KDA (per-key-channel gate) varlen decode
 * ``gdn_state_quantize_fp8`` / ``gdn_state_dequantize_fp8``  fp8 tile codec
@@ -84,6 +85,15 @@ class gdn_decode_paged_params(ctypes.Structure):
                 ("err_flags", _vp), ("pool", gdn_state_pool)]
 
 
+class gdn_prefill_paged_params(ctypes.Structure):
+    _fields_ = [("struct_size", _i32), ("B", _i32), ("total_tokens", _i32), ("H", _i32), ("HV", _i32),
+                ("K", _i32), ("V", _i32), ("in_dtype", _i32), ("out_dtype", _i32), ("index_dtype", _i32),
+                ("readout", _i32), ("use_qk_l2norm", _i32), ("page_size", _i32), ("scale", ctypes.c_float),
+                ("nnz", _i64), ("q", _vp), ("k", _vp), ("v", _vp), ("a", _vp), ("b", _vp), ("A_log", _vp),
+                ("dt_bias", _vp), ("cu_seqlens", _vp), ("page_indices", _vp), ("page_indptr", _vp),
+                ("last_page_len", _vp), ("out", _vp), ("err_flags", _vp), ("pool", gdn_state_pool)]
+
+
 class kda_decode_varlen_params(ctypes.Structure):
     _fields_ = [("struct_size", _i32), ("B", _i32), ("total_tokens", _i32), ("Hk", _i32),
                 ("HV", _i32), ("K", _i32), ("V", _i32), ("in_dtype", _i32), ("out_dtype", _i32),
@@ -104,13 +114,14 @@ def lib() -> ctypes.CDLL:
         L.gdn_decode_slots.argtypes = [ctypes.POINTER(gdn_decode_slots_params), _vp]
         L.gdn_decode_paged.argtypes = [ctypes.POINTER(gdn_decode_paged_params), _vp]
         L.kda_decode_varlen.argtypes = [ctypes.POINTER(kda_decode_varlen_params), _vp]
+        L.gdn_prefill_paged.argtypes = [ctypes.POINTER(gdn_prefill_paged_params), _vp]
         L.gdn_paged_decode_slots.argtypes = [_vp, _vp, _vp, _i32, _i64, _i32, _i64, _i32, _vp, _vp, _vp]
         L.gdn_state_quantize_fp8.argtypes = [_vp, _vp, _vp, _i64, _i32, _i32, _i32, _i32, _vp]
         L.gdn_state_dequantize_fp8.argtypes = [_vp, _vp, _vp, _i64, _i32, _i32, _i32, _i32, _vp]
         L.gdn_status_string.argtypes = [ctypes.c_int]
         L.gdn_status_string.restype = ctypes.c_char_p
         for f in ("gdn_decode_slots", "gdn_decode_paged", "kda_decode_varlen", "gdn_paged_decode_slots",
-                  "gdn_state_quantize_fp8", "gdn_state_dequantize_fp8"):
+                  "gdn_state_quantize_fp8", "gdn_state_dequantize_fp8", "gdn_prefill_paged"):
             getattr(L, f).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -310,6 +321,57 @@ def gdn_decode_paged(q, k, v, A_log, a, dt_bias, b, scale=None, output=None, use
     return out
 
 
+def gdn_prefill_paged(q, k, v, a, b, A_log, dt_bias, cu_seqlens, *, state_pool, page_indices, page_indptr,
+                      last_page_len, page_size, state_scales=None, state_layout="V_FIRST", block_v=64,
+                      scale=None, use_qk_l2norm=True, output=None, output_dtype=None, readout="working",
+                      err_flags=None):
+    """Append a varlen run of tokens to every paged sequence (prefill or
+    continued prefill); fresh sequences start from a zero state.
+
+    q, k [total, H, K]; v [total, HV, V]; a, b [total, HV]; A_log, dt_bias
+    [HV] fp32; cu_seqlens [B+1] int32; the CSR page table, whose
+    last_page_len counts the new tokens. Returns output [total, HV, V].
+    """
+    total, H, K = q.shape
+    HV, V = v.shape[1], v.shape[2]
+    B = cu_seqlens.numel() - 1
+    if page_size <= 0:
+        raise ValueError("prefill needs page_size")
+    _expect(k, (total, H, K), "k")
+    _expect(v, (total, HV, V), "v")
+    _expect(a, (total, HV), "a")
+    _expect(b, (total, HV), "b")
+    _expect(A_log, (HV,), "A_log")
+    _expect(dt_bias, (HV,), "dt_bias")
+    _expect(page_indptr, (B + 1,), "page_indptr")
+    _expect(last_page_len, (B,), "last_page_len")
+    if cu_seqlens.dtype != torch.int32 or page_indices.dim() != 1:
+        raise ValueError("cu_seqlens must be int32 and page_indices 1-D")
+    if A_log.dtype != torch.float32 or dt_bias.dtype != torch.float32:
+        raise ValueError("A_log and dt_bias must be float32")
+    if len({x.dtype for x in (q, k, v, a, b)}) != 1:
+        raise ValueError("q, k, v, a, b must share one dtype")
+    out_dt = output_dtype or (output.dtype if output is not None else q.dtype)
+    out = _out(output, (total, HV, V), out_dt, q)
+    prm = gdn_prefill_paged_params()
+    prm.struct_size = ctypes.sizeof(gdn_prefill_paged_params)
+    prm.B, prm.total_tokens, prm.H, prm.HV, prm.K, prm.V = B, total, H, HV, K, V
+    prm.in_dtype, prm.out_dtype = _io_dtype(q), _io_dtype(out)
+    prm.index_dtype = _same_index_dtype(page_indices, page_indptr, last_page_len)
+    prm.readout = _READOUTS[readout]
+    prm.use_qk_l2norm = int(bool(use_qk_l2norm))
+    prm.page_size = int(page_size)
+    prm.scale = 0.0 if scale is None else float(scale)
+    prm.nnz = page_indices.numel()
+    prm.q, prm.k, prm.v, prm.a, prm.b = _ptr(q), _ptr(k), _ptr(v), _ptr(a), _ptr(b)
+    prm.A_log, prm.dt_bias, prm.cu_seqlens = _ptr(A_log), _ptr(dt_bias), _ptr(cu_seqlens)
+    prm.page_indices, prm.page_indptr, prm.last_page_len = _ptr(page_indices), _ptr(page_indptr), _ptr(last_page_len)
+    prm.out, prm.err_flags = _ptr(out), _ptr(err_flags)
+    prm.pool = _pool(state_pool, state_scales, state_layout, block_v, K, V, HV)
+    _check(lib().gdn_prefill_paged(ctypes.byref(prm), _stream(q)), "gdn_prefill_paged")
+    return out
+
+
 def gdn_paged_decode_slots(page_indices, page_indptr, last_page_len, num_pages, page_size=0,
                            slots_out=None, err_flags=None):
     """(read_page, write_page) int64 rows [B, 2] of a paged decode step."""
@@ -392,6 +454,6 @@ def gdn_state_dequantize_fp8(codes, scales, *, block_v=64, layout="V_FIRST", out
     return out
 
 
-__all__ = ["gdn_decode_slots", "gdn_decode_paged", "gdn_paged_decode_slots", "kda_decode_varlen",
+__all__ = ["gdn_decode_slots", "gdn_decode_paged", "gdn_prefill_paged", "gdn_paged_decode_slots", "kda_decode_varlen",
            "gdn_state_quantize_fp8", "gdn_state_dequantize_fp8", "gdn_status_string", "GDNError",
            "LIB_PATH", "lib"]

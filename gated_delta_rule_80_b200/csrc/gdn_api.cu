@@ -339,6 +339,42 @@ int gdn_decode_paged(const gdn_decode_paged_params* p, gdn_stream_t stream) {
   return launch_step<GATE_SCALAR, IDX_PAGED>(k, p->pool, p->K, p->B, reinterpret_cast<cudaStream_t>(stream));
 }
 
+int gdn_prefill_paged(const gdn_prefill_paged_params* p, gdn_stream_t stream) {
+  if (p == nullptr || p->struct_size != static_cast<int32_t>(sizeof(gdn_prefill_paged_params)))
+    return GDN_ERR_INVALID_ARG;
+  if (p->B < 0 || p->total_tokens < 0 || p->H <= 0 || p->HV <= 0 || p->HV % p->H != 0 || p->nnz < 0)
+    return GDN_ERR_INVALID_ARG;
+  if (p->page_size <= 0) return GDN_ERR_INVALID_ARG;
+  if (!head_dim_ok(p->K) || !head_dim_ok(p->V)) return GDN_ERR_INVALID_ARG;
+  if (!io_dtype_ok(p->in_dtype) || !io_dtype_ok(p->out_dtype)) return GDN_ERR_INVALID_ARG;
+  if (p->index_dtype != GDN_I32 && p->index_dtype != GDN_I64) return GDN_ERR_INVALID_ARG;
+  if (p->readout != GDN_READOUT_WORKING && p->readout != GDN_READOUT_STORED) return GDN_ERR_INVALID_ARG;
+  if (const int rc = check_pool(p->pool, p->V)) return rc;
+  if (p->B == 0 || p->total_tokens == 0) return GDN_OK;
+  const uintptr_t es = io_size(p->in_dtype), is = index_size(p->index_dtype);
+  if (!ptrs_ok({p->q, p->k, p->v, p->out},
+               {{p->a, es}, {p->b, es}, {p->A_log, 4}, {p->dt_bias, 4}, {p->cu_seqlens, 4},
+                {p->page_indices, is}, {p->page_indptr, is}, {p->last_page_len, is}}))
+    return GDN_ERR_INVALID_ARG;
+  if (const int rc = select_device(p->pool.data)) return rc;
+
+  StepParams k{};
+  k.q = p->q; k.k = p->k; k.v = p->v; k.gate = p->a; k.beta = p->b;
+  k.A_log = p->A_log; k.dt_bias = p->dt_bias;
+  k.pool = p->pool.data; k.scales = p->pool.scales;
+  k.idx = p->page_indices; k.indptr = p->page_indptr; k.lastlen = p->last_page_len; k.cu = p->cu_seqlens;
+  k.out = p->out; k.err = p->err_flags;
+  k.num_slots = p->pool.num_slots; k.nnz = p->nnz;
+  k.B = p->B; k.T = 0; k.H = p->H; k.HV = p->HV; k.V = p->V;
+  k.total_tokens = p->total_tokens;
+  k.page_size = p->page_size;
+  k.scale = default_scale(p->scale, p->K);
+  k.flags = (p->in_dtype == GDN_BF16 ? F_IN_BF16 : 0) | (p->out_dtype == GDN_BF16 ? F_OUT_BF16 : 0) |
+            (p->index_dtype == GDN_I64 ? F_IDX64 : 0) | (p->use_qk_l2norm ? F_L2NORM : 0) | F_VARLEN |
+            (p->readout == GDN_READOUT_STORED ? F_READOUT_STORED : 0);
+  return launch_step<GATE_SCALAR, IDX_PAGED>(k, p->pool, p->K, p->B, reinterpret_cast<cudaStream_t>(stream));
+}
+
 int gdn_paged_decode_slots(const void* page_indices, const void* page_indptr, const void* last_page_len,
                            int32_t index_dtype, int64_t nnz, int32_t B, int64_t num_pages, int32_t page_size,
                            int64_t* slots_out, int32_t* err_flags, gdn_stream_t stream) {

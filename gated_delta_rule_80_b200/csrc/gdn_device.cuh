@@ -52,6 +52,7 @@ struct StepParams {
   const void* idx;      // slots: state_indices [B]; paged: page_indices [nnz]
   const void* indptr;   // paged: page_indptr [B+1]; varlen: cu_seqlens [B+1] int32
   const void* lastlen;  // paged: last_page_len [B]
+  const int32_t* cu;    // paged prefill: cu_seqlens [B+1]
   const int64_t* rows;  // paged: precomputed (read, write) [B, 2] or null
   void* out;            // [tok, HV, V]
   int32_t* err;         // optional
@@ -282,6 +283,8 @@ struct Unit {
   int status;
   int err;
   int64_t p0, L;     // paged suffix: first CSR position and tokens of the sequence
+  int T;             // paged suffix: tokens of the run
+  bool fresh;        // paged prefill of a sequence with no earlier token: S starts at 0
 };
 
 __device__ __forceinline__ int64_t ld_index(const void* base, int64_t i, bool i64) {
@@ -311,35 +314,39 @@ __device__ __forceinline__ void resolve_page_rows(const void* indices, const voi
   write = w;
 }
 
-// The last T tokens of a paged sequence: a page holds the state after its
+// The last n tokens of a paged sequence: a page holds the state after its
 // last token, so with L = (pages - 1) * page_size + last_page_len the state
-// is read from the page of position L-T-1 and the final state goes to the
-// last page (pages filled inside the suffix are written by the kernel's
-// token loop, see suffix_snapshot_page).
-__device__ __forceinline__ void resolve_suffix(const StepParams& p, int b, Unit& u) {
+// is read from the page of position L-n-1 and the final state goes to the
+// last page (pages filled inside the run are written by the kernel's token
+// loop, see suffix_snapshot_page). With allow_fresh, a sequence with no
+// earlier token (L == n) starts from a zero state.
+__device__ __forceinline__ void resolve_suffix(const StepParams& p, int b, int n, bool allow_fresh, Unit& u) {
   const bool i64 = (p.flags & F_IDX64) != 0;
   u.src = u.dst = -1;
+  u.T = n;
   const int64_t p0 = ld_index(p.indptr, b, i64);
   const int64_t p1 = ld_index(p.indptr, b + 1, i64);
   const int64_t len = ld_index(p.lastlen, b, i64);
   if (p0 < 0 || p1 > p.nnz) { u.err |= E_PAGE_RANGE; return; }
   if (p1 <= p0 || len < 1 || len > p.page_size) { u.err |= E_PAGE_TABLE; return; }
   const int64_t L = (p1 - p0 - 1) * p.page_size + len;
-  if (L < p.T + 1) { u.err |= E_PAGE_TABLE; return; }
-  const int64_t r = ld_index(p.idx, p0 + (L - p.T - 1) / p.page_size, i64);
+  const bool fresh = allow_fresh && L == n;
+  if (!fresh && L < n + 1) { u.err |= E_PAGE_TABLE; return; }
+  const int64_t r = fresh ? 0 : ld_index(p.idx, p0 + (L - n - 1) / p.page_size, i64);
   const int64_t w = ld_index(p.idx, p1 - 1, i64);
   if (r < 0 || r >= p.num_slots || w < 0 || w >= p.num_slots) { u.err |= E_PAGE_RANGE; return; }
-  u.src = r;
+  u.src = fresh ? -1 : r;
   u.dst = w;
   u.p0 = p0;
   u.L = L;
+  u.fresh = fresh;
 }
 
-// Page that receives the state after suffix token t (not the last one), or
-// -1: the page whose last position is L-T+t, when that position closes a page.
+// Page that receives the state after run token t (not the last one), or -1:
+// the page whose last position is L-n+t, when that position closes a page.
 __device__ __forceinline__ int64_t suffix_snapshot_page(const StepParams& p, const Unit& u, int t) {
-  const int64_t pos = u.L - p.T + t;
-  if (t >= p.T - 1 || (pos % p.page_size) != p.page_size - 1) return -1;
+  const int64_t pos = u.L - u.T + t;
+  if (t >= u.T - 1 || (pos % p.page_size) != p.page_size - 1) return -1;
   return ld_index(p.idx, u.p0 + pos / p.page_size, (p.flags & F_IDX64) != 0);
 }
 
@@ -350,6 +357,8 @@ __device__ __forceinline__ Unit resolve_unit(const StepParams& p, int b) {
   u.err = 0;
   u.p0 = 0;
   u.L = 0;
+  u.T = 0;
+  u.fresh = false;
   const bool i64 = (p.flags & F_IDX64) != 0;
   if constexpr (IDX == IDX_SLOTS) {
     if (p.flags & F_VARLEN) {
@@ -369,11 +378,24 @@ __device__ __forceinline__ Unit resolve_unit(const StepParams& p, int b) {
     u.src = u.dst = s;
     if (s < 0) u.status = U_PAD;
     else if (s >= p.num_slots) { u.status = U_PAD; u.err |= E_SLOT_RANGE; }
+  } else if (p.flags & F_VARLEN) {
+    // prefill: a varlen run appended to the sequence (see resolve_suffix)
+    const int32_t* cu = reinterpret_cast<const int32_t*>(p.cu);
+    u.tok0 = cu[b];
+    u.tok1 = cu[b + 1];
+    if (u.tok0 < 0 || u.tok1 < u.tok0 || u.tok1 > p.total_tokens) {
+      u.err |= E_SEQLENS;
+      u.status = U_SKIP;
+      return u;
+    }
+    if (u.tok1 == u.tok0) return u;
+    resolve_suffix(p, b, u.tok1 - u.tok0, true, u);
+    if (u.err) u.status = U_PAD;
   } else if (p.T > 1) {
     // suffix of T tokens (see resolve_suffix)
     u.tok0 = b * p.T;
     u.tok1 = u.tok0 + p.T;
-    resolve_suffix(p, b, u);
+    resolve_suffix(p, b, p.T, false, u);
     if (u.err) u.status = U_PAD;
   } else {
     u.tok0 = b;

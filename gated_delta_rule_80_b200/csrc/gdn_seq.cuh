@@ -137,14 +137,19 @@ step_seq(const StepParams p) {
   // ---- state tile loads
   using SV = StateVec<SDT, (VB >= 16 ? VB : 8)>;
   const int64_t head_bytes = (int64_t)K * V * ST::BYTES;
-  const char* src = reinterpret_cast<const char*>(p.pool) + (u.src * p.HV + hv) * head_bytes;
+  const char* src = reinterpret_cast<const char*>(p.pool) + ((u.fresh ? 0 : u.src) * p.HV + hv) * head_bytes;
   float S[NR][EPL];
   // element offset (within the head) of vector jj of this thread
   auto vec_off = [&](int jj) -> int64_t {
     if constexpr (VF) return (int64_t)(v0 + row0 + jj * RPW) * K + kofs;
     else return (int64_t)(g + RG * jj) * V + v0 + c0;
   };
-  if constexpr (VB >= 8) {
+  if (u.fresh) {  // a paged prefill with no earlier token: S starts at zero
+#pragma unroll
+    for (int jj = 0; jj < NR; ++jj)
+#pragma unroll
+      for (int e = 0; e < EPL; ++e) S[jj][e] = 0.0f;
+  } else if constexpr (VB >= 8) {
     typename SV::T raw[NR];
 #pragma unroll
     for (int jj = 0; jj < NR; ++jj) raw[jj] = SV::load(src + vec_off(jj) * ST::BYTES);
@@ -164,7 +169,7 @@ step_seq(const StepParams p) {
   const int n_scale = p.V / 64;
   const int stile = v0 / 64;  // fp8: this CTA's scale tile
   if constexpr (SDT == ST_FP8) {
-    const float sc = p.scales[(u.src * p.HV + hv) * n_scale + stile];
+    const float sc = u.fresh ? 0.0f : p.scales[(u.src * p.HV + hv) * n_scale + stile];
 #pragma unroll
     for (int jj = 0; jj < NR; ++jj)
 #pragma unroll
@@ -440,7 +445,7 @@ step_seq(const StepParams p) {
       if (writer) st_out1(p.out, ((int64_t)tok * p.HV + hv) * V + out_col, o_mine, out_bf16);
       if constexpr (IDX == IDX_PAGED) {
         // a page that fills inside a multi-token suffix keeps this state
-        if (p.T > 1) {
+        if (u.T > 1) {
           const int64_t page = suffix_snapshot_page(p, u, tok - u.tok0);
           if (page >= p.num_slots) {
             if (threadIdx.x == 0) raise_err(p.err, E_PAGE_RANGE);

@@ -200,6 +200,44 @@ typedef struct gdn_decode_paged_params {
 
 int gdn_decode_paged(const gdn_decode_paged_params* p, gdn_stream_t stream);
 
+/* Prefill (or continued prefill) on a paged pool: append a varlen run of
+ * tokens to every sequence. Sequence b gets n = cu_seqlens[b+1] - cu_seqlens[b]
+ * new tokens, the last n of its L = (pages - 1) * page_size + last_page_len
+ * tokens (the page table already includes them). The run is the scan of
+ * single steps over its tokens. The state starts at zero when the sequence
+ * has no earlier token (L == n), else it is read from the page of position
+ * L-n-1; every page that fills inside the run receives the state after its
+ * last token and the final state goes to the last page. n == 0 leaves the
+ * sequence untouched.
+ *  q, k [total_tokens, H, K]; v [total_tokens, HV, V]; a, b [total_tokens, HV]
+ *  (in_dtype); A_log, dt_bias [HV] fp32; cu_seqlens [B+1] int32;
+ *  page_indices [nnz], page_indptr [B+1], last_page_len [B] (index_dtype);
+ *  out [total_tokens, HV, V] (out_dtype). page_size > 0 is required. */
+typedef struct gdn_prefill_paged_params {
+  int32_t struct_size; /* sizeof(gdn_prefill_paged_params) */
+  int32_t B, total_tokens, H, HV, K, V;
+  int32_t in_dtype, out_dtype, index_dtype, readout, use_qk_l2norm;
+  int32_t page_size;
+  float scale;
+  int64_t nnz;
+  const void* q;
+  const void* k;
+  const void* v;
+  const void* a;
+  const void* b;
+  const float* A_log;
+  const float* dt_bias;
+  const int32_t* cu_seqlens;
+  const void* page_indices;
+  const void* page_indptr;
+  const void* last_page_len;
+  void* out;
+  int32_t* err_flags;  /* may be NULL */
+  gdn_state_pool pool;
+} gdn_prefill_paged_params;
+
+int gdn_prefill_paged(const gdn_prefill_paged_params* p, gdn_stream_t stream);
+
 /* Resolve the (read_page, write_page) rows of a paged decode once per step,
  * to be shared by every layer's gdn_decode_paged call.
  *  page_indices [nnz], page_indptr [B+1], last_page_len [B] (index_dtype);

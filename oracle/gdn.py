@@ -400,6 +400,61 @@ def gdn_decode_paged(q, k, v, a, b, A_log, dt_bias, state_pool, page_indices, pa
     return out, writes
 
 
+def gdn_prefill_paged(q, k, v, a, b, A_log, dt_bias, cu_seqlens, state_pool, page_indices, page_indptr,
+                      last_page_len, page_size, *, state_dtype="f32", state_scales=None, block_v=64,
+                      scale=None, use_qk_l2norm=True, readout_mode="working", layout="V_FIRST",
+                      units=None):
+    """Append varlen token runs to paged sequences (prefill, or continued prefill).
+
+    Sequence bb gets n = cu_seqlens[bb+1] - cu_seqlens[bb] new tokens, the
+    last n of its L tokens (L from the page table). The sequence is the scan
+    of single steps over them (Circuit.LLM.Mixer, scanMixer /
+    gatedDeltaPrefill). The state starts from zero when the sequence has no
+    earlier token (L == n), else from the page of position L-n-1; every page
+    that fills inside the run keeps the state after its last token, the
+    final state goes to the last page (``suffix_pages``). q, k: [total, H,
+    K]; v: [total, HV, V]; a, b: [total, HV].
+    Returns (out [total, HV, V], writes keyed by (page, hv)).
+    """
+    q = np.asarray(q, np.float64); k = np.asarray(k, np.float64)
+    v = np.asarray(v, np.float64); a = np.asarray(a, np.float64); b = np.asarray(b, np.float64)
+    total, H, K = q.shape
+    HV, V = v.shape[1], v.shape[2]
+    sc = _scale_of(scale, K)
+    B = len(cu_seqlens) - 1
+    out = np.full((total, HV, V), np.nan) if units is not None else np.zeros((total, HV, V))
+    writes = {}
+    todo = [(bb, hv) for bb in range(B) for hv in range(HV)] if units is None else list(units)
+    for (bb, hv) in todo:
+        bos, eos = int(cu_seqlens[bb]), int(cu_seqlens[bb + 1])
+        n = eos - bos
+        if n == 0:
+            continue
+        p0, p1 = int(page_indptr[bb]), int(page_indptr[bb + 1])
+        L = (p1 - p0 - 1) * page_size + int(last_page_len[bb])
+        if L == n:       # a fresh sequence: the state starts at zero
+            S0 = np.zeros((K, V))
+            snaps = [(t, int(page_indices[p0 + t // page_size])) for t in range(n - 1)
+                     if t % page_size == page_size - 1]
+            final = int(page_indices[p1 - 1])
+        else:
+            read, snaps, final = suffix_pages(page_indices, page_indptr, last_page_len, page_size, n, bb)
+            S0 = load_state(state_pool[read, hv], layout, state_dtype,
+                            None if state_scales is None else state_scales[read, hv], block_v)
+        h = key_head_of(hv, H, HV)
+        toks = []
+        for t in range(bos, eos):
+            qh, kh = prepare_qk(q[t, h], k[t, h], sc, use_qk_l2norm)
+            toks.append((qh, kh, v[t, hv], gdn_alpha(A_log[hv], a[t, hv], dt_bias[hv]), beta_of(b[t, hv])))
+        snap_at = dict(snaps)
+        for t, (o, payload) in enumerate(step_unit(S0, toks, state_dtype, readout_mode, block_v)):
+            out[bos + t, hv, :] = o
+            if t in snap_at:
+                writes[(snap_at[t], hv)] = store_state(payload, layout, state_dtype)
+        writes[(final, hv)] = store_state(payload, layout, state_dtype)
+    return out, writes
+
+
 def paged_decode_slots(page_indices, page_indptr, last_page_len):
     """[B, 2] int64 rows (read_page, write_page) for every sequence of the table."""
     B = len(page_indptr) - 1

@@ -30,6 +30,18 @@ BF16_OUT = 2.0 ** -8
 # a handful of such codes per tile, 1e-2 of the slice's max bounds it; the
 # output is then also checked against the stored state it was read from.
 TOL_FP8_STORED = 1e-2
+# fp8 state over a run of several tokens: the state is re-encoded after every
+# token, so a code that lands on the neighbouring E4M3 value on one side
+# (an fp32 rounding difference at a rounding boundary) is carried into the
+# later tokens' outputs; the same one-step bound applies. The stored codes
+# are still held to one step and >= 99.9% identical.
+TOL_FP8_RUN = 1e-2
+
+
+def out_tol(state_dtype, readout, multi_token):
+    if state_dtype == "fp8_e4m3" and (readout == "stored" or multi_token):
+        return TOL_FP8_RUN
+    return TOL[state_dtype]
 
 
 def dev(x: np.ndarray, dtype=None):
@@ -178,9 +190,8 @@ def gdn_slots_case(seed, B, T, H, HV, K, V, num_slots, layout="V_FIRST", state_d
         scale=scale, use_qk_l2norm=use_qk_l2norm, readout_mode=readout, num_slots=num_slots,
         units=units)
     todo = [(b, hv) for b in range(B) for hv in range(HV)] if units is None else units
-    tol = TOL_FP8_STORED if (state_dtype == "fp8_e4m3" and readout == "stored") else TOL[state_dtype]
     res["out_err"] = check_outputs(res["out"], ref_out, todo, lambda x, b, hv: x[b, :, hv, :],
-                                   tol, out_dtype)
+                                   out_tol(state_dtype, readout, T > 1), out_dtype)
     if state_dtype == "fp8_e4m3" and readout == "stored":
         check_stored_readout(res["out"], t, idx, after, sc_after, todo, layout, scale, use_qk_l2norm,
                              num_slots, block_v)
@@ -238,7 +249,7 @@ def gdn_paged_case(seed, B, H, HV, K, V, page_size, max_len, n_share, share_page
         readout_mode=readout, units=todo, page_size=page_size, layout=layout)
     out_h = host(out)
     res["out_err"] = check_outputs(out_h, ref_out, todo, lambda x, b, hv: x[b, :, hv, :],
-                                   TOL[state_dtype], out_dtype)
+                                   out_tol(state_dtype, readout, T > 1), out_dtype)
     # written pages: compare the sampled units; every other page must be bit-identical
     write_pages = sorted({pg for (pg, _) in writes}) if units is None else sorted(set(rows[:, 1].tolist()))
     wp = torch.tensor(write_pages, device="cuda")
@@ -254,6 +265,54 @@ def gdn_paged_case(seed, B, H, HV, K, V, page_size, max_len, n_share, share_page
         assert torch.equal(scales[keep], sc_snap[keep])
     res["write_pages"] = write_pages
     res["writes"] = writes
+    return res
+
+
+# ----------------------------------------------------------------------------
+# paged prefill case
+# ----------------------------------------------------------------------------
+
+def gdn_prefill_case(seed, B, H, HV, K, V, page_size, max_len, state_dtype="f32", in_dtype="bf16",
+                     out_dtype="f32", index_dtype="i32", layout="V_FIRST", fresh_every=2):
+    pt = W.paged_table(seed, B, page_size, max_len, 0, 0).cast(index_dtype)
+    cu = W.prefill_runs(seed, pt.seq_lens.tolist(), fresh_every)
+    total = int(cu[-1])
+    t = W.varlen_gdn_tokens(seed, total, H, HV, K, V, in_dtype)
+    reads = set()
+    for bb in range(B):
+        n = int(cu[bb + 1] - cu[bb])
+        if 0 < n < int(pt.seq_lens[bb]):
+            reads.add(O.suffix_pages(pt.page_indices, pt.page_indptr, pt.last_page_len, page_size, n, bb)[0])
+    pool, scales = W.device_pool(seed, pt.num_pages, HV, K, V, layout, state_dtype, exact_slots=sorted(reads))
+    snap = pool.clone()
+    sc_snap = scales.clone() if scales is not None else None
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out = G.gdn_prefill_paged(
+        dev_in(t["q"], in_dtype), dev_in(t["k"], in_dtype), dev_in(t["v"], in_dtype), dev_in(t["a"], in_dtype),
+        dev_in(t["b"], in_dtype), dev(t["A_log"]), dev(t["dt_bias"]), dev(cu), state_pool=pool,
+        page_indices=dev(pt.page_indices), page_indptr=dev(pt.page_indptr), last_page_len=dev(pt.last_page_len),
+        page_size=page_size, state_scales=scales, state_layout=layout, output_dtype=W.torch_dtype(out_dtype),
+        err_flags=err)
+    torch.cuda.synchronize()
+    states, sc = W.host_pool(seed, sorted(reads), HV, K, V, layout, state_dtype)
+    ref_out, writes = O.gdn_prefill_paged(t["q"], t["k"], t["v"], t["a"], t["b"], t["A_log"], t["dt_bias"], cu,
+                                          states, pt.page_indices, pt.page_indptr, pt.last_page_len, page_size,
+                                          state_dtype=state_dtype, state_scales=sc, layout=layout)
+    units = [(bb, hv) for bb in range(B) for hv in range(HV)]
+    res = dict(err=int(err.item()), cu=cu, table=pt)
+    res["out_err"] = check_outputs(host(out), ref_out, units, lambda x, bb, hv: x[int(cu[bb]):int(cu[bb + 1]), hv, :],
+                                   out_tol(state_dtype, "working", True), out_dtype)
+    write_pages = sorted({pg for (pg, _) in writes})
+    wp = torch.tensor(write_pages, device="cuda")
+    pos = {pg: i for i, pg in enumerate(write_pages)}
+    res["state_err"] = check_state(pool_host(pool[wp]), scales[wp].cpu().numpy() if scales is not None else None,
+                                   {(pos[pg], hv): w for (pg, hv), w in writes.items()}, state_dtype, layout)
+    keep = torch.ones(pt.num_pages, dtype=torch.bool, device="cuda")
+    keep[wp] = False
+    assert torch.equal(pool[keep], snap[keep]), "a page the runs do not fill changed"
+    if scales is not None:
+        assert torch.equal(scales[keep], sc_snap[keep])
+    res["write_pages"] = write_pages
     return res
 
 
@@ -293,7 +352,7 @@ def kda_case(seed, B, Hk, HV, K, V, num_slots, max_len, layout="K_FIRST", state_
     res = dict(out=out_h, err=int(err.item()), writes=writes, pool_before=before, pool_after=after, cu=cu)
     res["out_err"] = check_outputs(out_h, ref_out, units,
                                    lambda x, b, hv: x[int(cu[b]):int(cu[b + 1]), hv, :],
-                                   TOL[state_dtype], out_dtype)
+                                   out_tol(state_dtype, readout, True), out_dtype)
     res["state_err"] = check_state(after, sc_after, writes, state_dtype, layout)
     check_untouched(before, after, writes.keys(), sc_before, sc_after)
     return res

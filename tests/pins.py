@@ -525,4 +525,40 @@ def pin_paged_suffix_equals_single_steps():
             assert np.array_equal(p[pg], pool[pg])
 
 
+def pin_prefill_matches_decode_and_split():
+    """A fresh prefill of L tokens from a zero state equals: (a) the slot
+    decode of the same L tokens from a zero state, with the page snapshots
+    equal to the states after each page's last token; (b) a prefill of the
+    first n tokens followed by a continued prefill of the rest."""
+    ps, H, HV, K, V = 4, 1, 2, 4, 4
+    L = 11
+    ind = [3, 0, 5]                    # pages of positions 0-3, 4-7, 8-10
+    t = _tiny_tokens(91, 1, L, H, HV, K, V)
+    tok = {n: t[n][0] for n in ("q", "k", "v", "a", "b")}
+    pool = _tiny_pool(92, 6, HV, K, V).astype(np.float64)
+    out, writes = O.gdn_prefill_paged(tok["q"], tok["k"], tok["v"], tok["a"], tok["b"], t["A_log"], t["dt_bias"],
+                                      [0, L], pool, ind, [0, 3], [3], ps)
+    zero = np.zeros((1, HV, V, K))
+    ref_out, _ = O.gdn_decode_slots(t["q"], t["k"], t["v"], t["a"], t["b"], t["A_log"], t["dt_bias"], zero, [0])
+    assert np.allclose(out, ref_out[0], rtol=0, atol=1e-12)
+    for n_pref, page in ((4, 3), (8, 0), (11, 5)):
+        _, w = O.gdn_decode_slots(t["q"][:, :n_pref], t["k"][:, :n_pref], t["v"][:, :n_pref], t["a"][:, :n_pref],
+                                  t["b"][:, :n_pref], t["A_log"], t["dt_bias"], zero, [0])
+        for hv in range(HV):
+            assert np.allclose(writes[(page, hv)][0], w[(0, hv)][0], rtol=0, atol=1e-6)
+    assert {pg for (pg, _) in writes} == {3, 0, 5}
+    # split: 6 tokens (pages 3 and half of 0), then the remaining 5
+    o1, w1 = O.gdn_prefill_paged(*(tok[n][:6] for n in ("q", "k", "v", "a", "b")), t["A_log"], t["dt_bias"],
+                                 [0, 6], pool, ind[:2], [0, 2], [2], ps)
+    p = pool.copy()
+    for (pg, hv), (st, _) in w1.items():
+        p[pg, hv] = st
+    o2, w2 = O.gdn_prefill_paged(*(tok[n][6:] for n in ("q", "k", "v", "a", "b")), t["A_log"], t["dt_bias"],
+                                 [0, 5], p, ind, [0, 3], [3], ps)
+    assert np.allclose(np.concatenate([o1, o2]), out, rtol=0, atol=1e-6)
+    for key in writes:
+        got = w2[key][0] if key in w2 else w1[key][0]
+        assert np.allclose(got, writes[key][0], rtol=0, atol=1e-6), key
+
+
 ALL_PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]

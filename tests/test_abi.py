@@ -31,7 +31,7 @@ def declared_functions():
 
 def test_every_declared_symbol_is_exported(lib):
     names = declared_functions()
-    assert {"gdn_decode_slots", "gdn_decode_paged", "gdn_paged_decode_slots", "kda_decode_varlen",
+    assert {"gdn_decode_slots", "gdn_decode_paged", "gdn_paged_decode_slots", "kda_decode_varlen", "gdn_prefill_paged",
             "gdn_state_quantize_fp8", "gdn_state_dequantize_fp8", "gdn_status_string"} <= set(names)
     for n in names:
         assert hasattr(lib, n), f"{n} is declared in include/gdn.h but not exported"
@@ -42,6 +42,7 @@ STRUCTS = {
     "gdn_decode_slots_params": G.gdn_decode_slots_params,
     "gdn_decode_paged_params": G.gdn_decode_paged_params,
     "kda_decode_varlen_params": G.kda_decode_varlen_params,
+    "gdn_prefill_paged_params": G.gdn_prefill_paged_params,
 }
 
 

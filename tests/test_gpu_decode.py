@@ -8,8 +8,8 @@ import torch
 
 import gated_delta_rule_80_b200 as G
 import workloads as W
-from gdn_cases import (check_outputs, dev, dev_in, gdn_paged_case, gdn_slots_case, host, kda_case,
-                       pool_host, slice_rel_err)
+from gdn_cases import (check_outputs, dev, dev_in, gdn_paged_case, gdn_prefill_case, gdn_slots_case, host,
+                       kda_case, pool_host, slice_rel_err)
 from oracle import formats
 from oracle import gdn as O
 
@@ -423,3 +423,22 @@ def test_kda_head_dim_256(layout):
 def test_paged_head_dim_256():
     gdn_paged_case(65, B=5, H=1, HV=2, K=256, V=256, page_size=8, max_len=40, n_share=2, share_pages=1,
                    force_lens={0: 9})
+
+
+# ----------------------------------------------------------------------------
+# paged prefill (fresh and continued runs)
+# ----------------------------------------------------------------------------
+
+@pytest.mark.parametrize("state_dtype", ["f32", "bf16", "fp8_e4m3"])
+@pytest.mark.parametrize("layout", ["V_FIRST", "K_FIRST"])
+def test_prefill_paged(state_dtype, layout):
+    r = gdn_prefill_case(71, B=6, H=1, HV=2, K=128, V=128, page_size=8, max_len=45, state_dtype=state_dtype,
+                         layout=layout)
+    assert r["err"] == 0
+    assert int(r["cu"][-1] - r["cu"][-2]) == 0   # the last sequence appends nothing
+
+
+def test_prefill_paged_long_runs_int64():
+    r = gdn_prefill_case(72, B=3, H=2, HV=4, K=64, V=128, page_size=16, max_len=300, index_dtype="i64",
+                         fresh_every=1)
+    assert r["err"] == 0 and len(r["write_pages"]) >= 3

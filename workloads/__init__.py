@@ -119,6 +119,29 @@ def gdn_tokens(seed, B, T, H, HV, K, V, in_dtype="bf16", stream=0) -> Dict[str, 
     return d
 
 
+def varlen_gdn_tokens(seed, total, H, HV, K, V, in_dtype="bf16", stream=0) -> Dict[str, np.ndarray]:
+    """GDN token inputs on a varlen token axis: q, k [total,H,K]; v [total,HV,V];
+    a, b [total,HV]; A_log, dt_bias [HV] (fp32)."""
+    d = gdn_tokens(seed, 1, total, H, HV, K, V, in_dtype, stream)
+    return {n: (x[0] if n not in ("A_log", "dt_bias") else x) for n, x in d.items()}
+
+
+def prefill_runs(seed, lens, fresh_every=2):
+    """New-run lengths for prefill tests: every ``fresh_every``-th sequence is
+    fresh (the whole sequence is new), the others append U[1, L-1] tokens,
+    and the last one appends nothing. Returns cu_seqlens [B+1] int32."""
+    r = _rng(seed, _LENGTHS, 7)
+    n = []
+    for bb, L in enumerate(lens):
+        if bb == len(lens) - 1 and len(lens) > 2:
+            n.append(0)
+        elif bb % fresh_every == 0 or L < 2:
+            n.append(int(L))
+        else:
+            n.append(int(r.integers(1, L)))
+    return np.concatenate([[0], np.cumsum(n)]).astype(np.int32)
+
+
 def kda_tokens(seed, total, Hk, HV, K, V, in_dtype="bf16", stream=0) -> Dict[str, np.ndarray]:
     """q, k [total,Hk,K]; v [total,HV,V]; raw_gate [total,HV,K]; beta_logits
     [total,HV]; a_log [HV]; dt_bias [HV,K] (fp32)."""
