@@ -50,7 +50,7 @@ def parse():
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["b200", "reference"], default="b200")
-    ap.add_argument("--workload", choices=["slots", "paged", "kda", "fp8", "tiny"], default="slots")
+    ap.add_argument("--workload", choices=["slots", "paged", "kda", "fp8", "tiny", "prefill"], default="slots")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
@@ -353,12 +353,58 @@ class KdaRun:
                 f"{self.layout}")
 
 
+class PrefillRun:
+    """Paged prefill (the 'prefill' workload): 8 fresh sequences of 1024
+    tokens, page_size 64, HV=32, H=16, K=V=128, bf16 in/out, fp32 pages.
+    Steps rotate over 4 page sets."""
+
+    def __init__(self, w: W.Workload, rank: int):
+        import gated_delta_rule_80_b200 as G
+        self.G = G
+        seed = 5 + 1000 * rank
+        self.B, self.L, self.ps, self.H, self.HV, self.K, self.V = 8, 1024, 64, 16, 32, 128, 128
+        npg = self.L // self.ps
+        self.n_rot = 4
+        total = self.B * self.L
+        t = W.varlen_gdn_tokens(seed, total, self.H, self.HV, self.K, self.V, "bf16")
+        self.ins = [in_t(t[n], "bf16") for n in ("q", "k", "v", "a", "b")]
+        self.A_log, self.dt_bias = in_t(t["A_log"], "f32"), in_t(t["dt_bias"], "f32")
+        self.cu = torch.from_numpy(np.arange(self.B + 1, dtype=np.int32) * self.L).cuda()
+        self.num_pages = self.n_rot * self.B * npg
+        self.pool, _ = W.device_pool(seed, self.num_pages, self.HV, self.K, self.V, "V_FIRST", "f32")
+        perm = np.random.default_rng(seed).permutation(self.num_pages).astype(np.int32)
+        self.tables = []
+        for r in range(self.n_rot):
+            ind = perm[r * self.B * npg:(r + 1) * self.B * npg]
+            self.tables.append((torch.from_numpy(ind.copy()).cuda(),
+                                torch.from_numpy(np.arange(self.B + 1, dtype=np.int32) * npg).cuda(),
+                                torch.full((self.B,), self.ps, dtype=torch.int32, device="cuda")))
+        self.out = torch.empty((total, self.HV, self.V), dtype=torch.bfloat16, device="cuda")
+        self.tokens_per_step = total
+        tok_bytes = (2 * self.H * self.K + 2 * self.HV * self.V + 2 * self.HV) * 2
+        self.bytes_per_step = total * tok_bytes + self.B * npg * self.HV * self.K * self.V * 4 + self.HV * 8
+        self.l2_note = f"rotating {self.n_rot} disjoint page sets ({self.B * npg * 2 * self.n_rot} MiB written per cycle)"
+
+    def step(self, i):
+        pi, pp, pl = self.tables[i % self.n_rot]
+        q, k, v, a, b = self.ins
+        self.G.gdn_prefill_paged(q, k, v, a, b, self.A_log, self.dt_bias, self.cu, state_pool=self.pool,
+                                 page_indices=pi, page_indptr=pp, last_page_len=pl, page_size=self.ps,
+                                 output=self.out)
+
+    def describe(self):
+        return (f"paged GDN prefill: {self.B} fresh sequences x {self.L} tokens, page_size={self.ps}, "
+                f"H={self.H}, HV={self.HV}, K=V={self.K}, bf16 in/out, fp32 pages (one snapshot per page)")
+
+
 def make_run(name, rank):
-    w = W.WORKLOADS[name]
+    w = W.WORKLOADS.get(name)
     if name in ("slots", "fp8", "tiny"):
         return SlotsRun(w, rank)
     if name == "paged":
         return PagedRun(w, rank)
+    if name == "prefill":
+        return PrefillRun(None, rank)
     return KdaRun(w, rank)
 
 
