@@ -5,8 +5,8 @@ TEST INFRASTRUCTURE, NOT PRODUCT CODE. Only the tests, the smoke check of
 The CUDA library never calls it and shares no code with it: the two meet
 only through the seeded input generators in ``workloads``.
 
-The oracle computes in float64 (the fp8 tile codec in binary32, so that
-codes and scales are exactly reproducible) and follows the pages' literal
+The oracle computes in float64 (the fp8 tile codec and the int8_hadamard32
+codec in binary32, so that codes and scales are exactly reproducible) and follows the pages' literal
 step order; see ``oracle.gdn`` for the sources and for every reading of a
 point the pages leave open.
 
@@ -19,9 +19,15 @@ Parity status of each function:
   sequential == repeated single steps, and the paged and slot pool rules.
 * ``formats``: pinned by the OCP E4M3 format's defined points, by library
   conversions (torch bf16 and float8_e4m3fn casts) and by grid properties.
+  The int8_hadamard32 codec: its rotation by scipy's Sylvester Hadamard
+  matrix and by closed forms (constant and unit vectors, R R = I), its
+  rounding by ties-to-even points, its grouping by the page's statement (one
+  scale per key channel and 32 values) and its error by the bound that an
+  orthonormal rotation carries over from the rotated domain.
 * conventions the pages do not fix (parity unpinned): the L2-norm epsilon,
   the GQA head map ``hv // (HV // H)``, the KDA gate's use of the GDN form
-  per key channel, and the tile codec's scale formula.
+  per key channel, the tile codec's scale formula, and for int8_hadamard32
+  the Hadamard order and normalisation and the scale formula amax / 127.
 """
 
 from . import formats, gdn  # noqa: F401

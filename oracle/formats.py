@@ -27,11 +27,38 @@ Test infrastructure only (see ``oracle/__init__.py``).
   A tile whose ``amax`` is 0, or whose ``r`` overflows binary32 (amax below
   about 1.3e-36), is stored as scale 0 with all codes +0 and decodes to 0.
 
+* int8_hadamard32 codec: the ModelOpt linear-attention config page
+  (LinearAttentionConfig, and LinearAttentionDecodeConfig ``state_codec``)
+  says only that this decode codec fixes its scales to one key channel and
+  32 values, while ``block_v`` stays the execution tile width. The rest is
+  the plainest reading of the name, stated here once:
+
+      x     = S[k, 32 g : 32 g + 32]       (one key channel, 32 values)
+      y     = R x,  R = H32 / sqrt(32)     (H32 the Sylvester Hadamard matrix,
+                                            natural order; R is symmetric and
+                                            orthonormal, so R R = I)
+      amax  = max |y|;  s = amax / 127;  r = 1 / s      (binary32)
+      code  = clamp(rint(y * r), -127, 127) as int8     (binary32 product,
+                                                         ties to even)
+      x'    = R (code * s)                 (binary32 product, then R)
+
+  so the stored scale array is ``[V / 32, K]`` per state (group-major). R is
+  applied in binary32 by the butterfly of the fast Walsh-Hadamard transform:
+  stages of span 1, 2, 4, 8, 16, each turning the pair at (i, i + span),
+  ``i & span == 0``, into (a + b, a - b), then one product with the binary32
+  nearest to 1/sqrt(32) (bit pattern 0x3E3504F3, exactly a quarter of the
+  nearest binary32 to 1/sqrt(2)). Every codec decision is thereby a binary32
+  computation with one fixed rounding order. A group whose ``amax`` is 0, or
+  whose ``r`` overflows binary32, stores scale 0 and codes 0. For finite
+  inputs ``|y * r|`` stays below 127.5, so the clamp never changes a code.
+
 Every function here works on numpy arrays and uses numpy's IEEE binary32 and
 binary64 arithmetic; nothing is shared with the CUDA path.
 """
 
 from __future__ import annotations
+
+import math
 
 import numpy as np
 
@@ -183,3 +210,95 @@ def dequantize_state(codes_kv: np.ndarray, scales: np.ndarray, block_v: int) -> 
         out[:, j * block_v:(j + 1) * block_v] = dequantize_tile(
             codes[:, j * block_v:(j + 1) * block_v], scales[j])
     return out
+
+
+# ----------------------------------------------------------------------------
+# int8_hadamard32: one scale per key channel and 32 values, after a
+# Walsh-Hadamard rotation of the 32 values
+# ----------------------------------------------------------------------------
+
+H32 = 32
+INT8_CODE_MAX = 127
+INV_SQRT32_F32 = np.array([0x3E3504F3], dtype=np.uint32).view(np.float32)[0]
+
+
+def fwht32(x: np.ndarray) -> np.ndarray:
+    """Unnormalised 32-point Walsh-Hadamard transform along the last axis.
+
+    Natural (Sylvester) order, computed in the dtype of ``x`` by butterfly
+    stages of span 1, 2, 4, 8, 16: the pair (a, b) at positions (i, i + span)
+    with ``i & span == 0`` becomes (a + b, a - b).
+    """
+    y = np.array(x, copy=True)
+    if y.shape[-1] != H32:
+        raise ValueError("last axis must hold 32 values")
+    lead = y.shape[:-1]
+    span = 1
+    while span < H32:
+        y = y.reshape(lead + (H32 // (2 * span), 2, span))
+        a = y[..., 0, :].copy()
+        b = y[..., 1, :].copy()
+        y[..., 0, :] = a + b
+        y[..., 1, :] = a - b
+        y = y.reshape(lead + (H32,))
+        span *= 2
+    return y
+
+
+def hadamard32(x: np.ndarray) -> np.ndarray:
+    """The orthonormal rotation R = H32 / sqrt(32) along the last axis.
+
+    binary32 input: the binary32 butterflies, then one binary32 product with
+    the nearest binary32 to 1/sqrt(32). Any other input: float64 throughout.
+    """
+    x = np.asarray(x)
+    if x.dtype == np.float32:
+        return (fwht32(x) * INV_SQRT32_F32).astype(np.float32)
+    return fwht32(x.astype(np.float64)) * (1.0 / math.sqrt(32.0))
+
+
+def h32_scales(amax: np.ndarray):
+    """Per-group (s, r) in binary32 from the groups' amax; groups stored as
+    zeros get s = 0 and r = 0."""
+    amax = np.asarray(amax, dtype=np.float32)
+    with np.errstate(over="ignore", divide="ignore", invalid="ignore"):
+        s = (amax / np.float32(INT8_CODE_MAX)).astype(np.float32)
+        r = (np.float32(1.0) / s).astype(np.float32)
+    zero = ~(amax > 0) | ~np.isfinite(r)
+    return np.where(zero, np.float32(0), s).astype(np.float32), np.where(zero, np.float32(0), r).astype(np.float32)
+
+
+def int8_round(y: np.ndarray) -> np.ndarray:
+    """binary32 values -> int8 codes: nearest integer, ties to even, clamped
+    to [-127, 127]."""
+    return np.clip(np.rint(np.asarray(y, np.float64)), -INT8_CODE_MAX, INT8_CODE_MAX).astype(np.int8)
+
+
+def quantize_rotated_groups(y: np.ndarray):
+    """Rotated groups ``y [..., 32]`` (binary32) -> (codes int8 [..., 32], scales [...])."""
+    y = np.asarray(y, np.float32)
+    amax = np.max(np.abs(y), axis=-1)
+    s, r = h32_scales(amax)
+    codes = int8_round((y * r[..., None]).astype(np.float32))
+    return codes, s
+
+
+def quantize_state_h32(S_kv: np.ndarray):
+    """Encode a logical [K, V] state: codes int8 [K, V] (rotated groups in
+    place of the values) and scales [V / 32, K] binary32."""
+    S = np.asarray(S_kv, dtype=np.float32)
+    K, V = S.shape
+    if V % H32:
+        raise ValueError("V must be a multiple of 32")
+    y = hadamard32(S.reshape(K, V // H32, H32))
+    codes, s = quantize_rotated_groups(y)
+    return codes.reshape(K, V), np.ascontiguousarray(s.T)
+
+
+def dequantize_state_h32(codes_kv: np.ndarray, scales: np.ndarray) -> np.ndarray:
+    """Decode a logical [K, V] int8 code array with its [V / 32, K] scales -> binary32."""
+    codes = np.asarray(codes_kv, dtype=np.int8)
+    K, V = codes.shape
+    sc = np.asarray(scales, np.float32).T               # [K, V / 32]
+    yq = (codes.reshape(K, V // H32, H32).astype(np.float32) * sc[..., None]).astype(np.float32)
+    return hadamard32(yq).reshape(K, V)

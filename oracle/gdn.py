@@ -42,7 +42,8 @@ Readings where the pages are silent (each one is a convention, not a pin):
   unit: output 0, nothing written.
 * state storage per token: fp32 states keep full precision across a
   multi-token call (the oracle holds float64); bf16 states are rounded to
-  bf16 after every token; fp8 states are re-encoded after every token.
+  bf16 after every token; fp8 and int8_hadamard32 states are re-encoded
+  after every token.
   ``readout='working'`` reads ``o`` from the state before that rounding,
   ``'stored'`` after it.
 
@@ -61,7 +62,7 @@ from . import formats
 
 L2NORM_EPS = 1e-6
 LAYOUTS = ("K_FIRST", "V_FIRST")
-STATE_DTYPES = ("f32", "bf16", "fp8_e4m3")
+STATE_DTYPES = ("f32", "bf16", "fp8_e4m3", "int8_hadamard32")
 
 
 # ----------------------------------------------------------------------------
@@ -181,6 +182,9 @@ def load_state(stored2d, layout, state_dtype, scales=None, block_v=64):
         codes_kv = _to_kv(np.asarray(stored2d, np.uint8), layout)
         return formats.dequantize_state(codes_kv, np.asarray(scales, np.float32),
                                         block_v).astype(np.float64)
+    if state_dtype == "int8_hadamard32":
+        codes_kv = _to_kv(np.asarray(stored2d, np.int8), layout)
+        return formats.dequantize_state_h32(codes_kv, scales).astype(np.float64)
     raise ValueError(state_dtype)
 
 
@@ -188,7 +192,8 @@ def write_event(S, state_dtype, block_v=64):
     """Round a float64 state the way its storage does after one token.
 
     Returns (S_stored_as_float64, payload) where payload is what is written
-    to the pool: fp32 array, bf16 bits, or (codes, scales) for fp8.
+    to the pool: fp32 array, bf16 bits, or (codes, scales) for fp8 and
+    int8_hadamard32.
     """
     if state_dtype == "f32":
         s32 = S.astype(np.float32)
@@ -200,12 +205,16 @@ def write_event(S, state_dtype, block_v=64):
         codes, scales = formats.quantize_state(S.astype(np.float32), block_v)
         deq = formats.dequantize_state(codes, scales, block_v)
         return deq.astype(np.float64), (codes, scales)
+    if state_dtype == "int8_hadamard32":
+        codes, scales = formats.quantize_state_h32(S.astype(np.float32))
+        deq = formats.dequantize_state_h32(codes, scales)
+        return deq.astype(np.float64), (codes, scales)
     raise ValueError(state_dtype)
 
 
 def store_state(payload, layout, state_dtype):
     """Payload from ``write_event`` -> (stored 2-D array in the layout, scales or None)."""
-    if state_dtype == "fp8_e4m3":
+    if state_dtype in ("fp8_e4m3", "int8_hadamard32"):
         codes, scales = payload
         return _from_kv(codes, layout), scales
     return _from_kv(payload, layout), None
@@ -221,7 +230,7 @@ def step_unit(S0, tokens, state_dtype, readout_mode="working", block_v=64):
     ``S0``: float64 [K, V] (already decoded). ``tokens``: iterable of
     ``(q_hat, k_hat, v, alpha, beta)``. ``payload`` is what the pool would
     hold if the state were stored right then. fp32 states carry float64
-    between tokens (a stored copy is rounded once); bf16 and fp8 states pass
+    between tokens (a stored copy is rounded once); bf16 and coded states pass
     through their storage after every token (a write event).
     """
     S = S0
@@ -267,8 +276,9 @@ def gdn_decode_slots(q, k, v, a, b, A_log, dt_bias, state_pool, state_indices, *
     """GDN decode of B sequences with T tokens each against a slot pool.
 
     q, k: [B, T, H, K]; v: [B, T, HV, V]; a, b: [B, T, HV]; A_log, dt_bias:
-    [HV]; state_pool[slot, hv] -> stored 2-D state (f32 array, bf16 bits or
-    fp8 codes); state_scales[slot, hv] -> [V/block_v] (fp8); state_indices [B].
+    [HV]; state_pool[slot, hv] -> stored 2-D state (f32 array, bf16 bits,
+    fp8 or int8 codes); state_scales[slot, hv] -> [V/block_v] (fp8) or
+    [V/32, K] (int8_hadamard32); state_indices [B].
 
     Returns (out [B, T, HV, V] float64, writes) where writes maps
     (slot, hv) -> (stored 2-D array, scales or None). ``units`` restricts the
@@ -535,4 +545,25 @@ def state_dequantize_fp8(codes, scales, block_v, layout):
     for n in range(codes.shape[0]):
         kv = formats.dequantize_state(_to_kv(codes[n], layout), scales[n], block_v)
         out[n] = _from_kv(kv, layout)
+    return out
+
+
+def state_quantize_h32(src, layout):
+    """src [N, *2-D state in layout*] binary32 -> (codes int8 same shape, scales [N, V/32, K])."""
+    src = np.asarray(src, np.float32)
+    codes = np.zeros(src.shape, np.int8)
+    scales = []
+    for n in range(src.shape[0]):
+        c, s = formats.quantize_state_h32(_to_kv(src[n], layout))
+        codes[n] = _from_kv(c, layout)
+        scales.append(s)
+    K = _to_kv(src[0], layout).shape[0] if src.shape[0] else 0
+    return codes, (np.stack(scales) if scales else np.zeros((0, 0, K), np.float32))
+
+
+def state_dequantize_h32(codes, scales, layout):
+    codes = np.asarray(codes, np.int8)
+    out = np.zeros(codes.shape, np.float32)
+    for n in range(codes.shape[0]):
+        out[n] = _from_kv(formats.dequantize_state_h32(_to_kv(codes[n], layout), scales[n]), layout)
     return out

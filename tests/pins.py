@@ -561,4 +561,147 @@ def pin_prefill_matches_decode_and_split():
         assert np.allclose(got, writes[key][0], rtol=0, atol=1e-6), key
 
 
+# ----------------------------------------------------------------------------
+# int8_hadamard32 state codec (ModelOpt linear-attention config: one scale per
+# key channel and 32 values)
+# ----------------------------------------------------------------------------
+
+def pin_hadamard32_matches_scipy():
+    """R = H32 / sqrt(32) against scipy's Sylvester Hadamard matrix; R R = I."""
+    import scipy.linalg
+    Hs = scipy.linalg.hadamard(32).astype(np.float64) / math.sqrt(32.0)
+    R = formats.hadamard32(np.eye(32))            # row i is R e_i (R is symmetric)
+    assert np.allclose(R, Hs, rtol=0, atol=1e-15)
+    x = np.random.default_rng(80).standard_normal((3, 5, 32))
+    assert np.allclose(formats.hadamard32(x), x @ Hs.T, rtol=0, atol=1e-13)
+    assert np.allclose(formats.hadamard32(formats.hadamard32(x)), x, rtol=0, atol=1e-13)
+    x32 = x.astype(np.float32)
+    y32 = formats.hadamard32(x32)
+    assert y32.dtype == np.float32
+    assert np.allclose(y32, x32.astype(np.float64) @ Hs.T, rtol=0, atol=4e-6)
+
+
+def pin_hadamard32_closed_forms():
+    """R 1 = sqrt(32) e_0; R e_j has entries (-1)^popcount(i & j) / sqrt(32)."""
+    y = formats.hadamard32(np.ones(32))
+    assert abs(y[0] - math.sqrt(32.0)) < 1e-13 and np.all(np.abs(y[1:]) < 1e-13)
+    for j in (0, 1, 5, 17, 31):
+        e = np.zeros(32)
+        e[j] = 1.0
+        ref = np.array([(-1.0) ** bin(i & j).count("1") for i in range(32)]) / math.sqrt(32.0)
+        assert np.allclose(formats.hadamard32(e), ref, rtol=0, atol=1e-15), j
+    # 0x3E3504F3 is the binary32 nearest to 1/sqrt(32): its neighbours are farther
+    c = float(formats.INV_SQRT32_F32)
+    lo = float(np.nextafter(np.float32(c), np.float32(0)))
+    hi = float(np.nextafter(np.float32(c), np.float32(1)))
+    err = lambda z: abs(Fraction(z) ** 2 * 32 - 1)
+    assert err(c) < err(lo) and err(c) < err(hi)
+
+
+def pin_int8_rounding_points():
+    """With amax = 127 the scale is 1, and codes are the integers nearest to
+    the rotated values, ties to even."""
+    y = np.zeros(32, np.float32)
+    pts = [127.0, 2.5, -2.5, 3.5, 0.5, -0.5, 1.5, 126.5, -126.5, 0.49999997, -1.5000001, 64.0]
+    want = [127, 2, -2, 4, 0, 0, 2, 126, -126, 0, -2, 64]
+    y[:len(pts)] = pts
+    codes, s = formats.quantize_rotated_groups(y[None])
+    assert s[0] == np.float32(1.0)
+    assert codes[0, :len(want)].tolist() == want and not codes[0, len(want):].any()
+    # a group at a scale that is a power of two rounds the same way
+    codes2, s2 = formats.quantize_rotated_groups((y * np.float32(2.0 ** -9))[None])
+    assert s2[0] == np.float32(2.0 ** -9) and np.array_equal(codes2, codes)
+
+
+def pin_h32_codec_groups():
+    """One scale per key channel and 32 values: scales [V/32, K]; a state that
+    is nonzero in one key row, or in one 32-value group, sets only those scales."""
+    r = np.random.default_rng(81)
+    K, V = 6, 96
+    S = np.zeros((K, V), np.float32)
+    S[4] = r.standard_normal(V)
+    codes, sc = formats.quantize_state_h32(S)
+    assert sc.shape == (V // 32, K)
+    assert np.all(sc[:, 4] > 0) and not np.delete(sc, 4, axis=1).any()
+    assert not np.delete(codes, 4, axis=0).any()
+    S = np.zeros((K, V), np.float32)
+    S[:, 32:64] = r.standard_normal((K, 32))
+    codes, sc = formats.quantize_state_h32(S)
+    assert np.all(sc[1] > 0) and not sc[0].any() and not sc[2].any()
+    assert not codes[:, :32].any() and not codes[:, 64:].any()
+    # each group is the codec of its own 32 values
+    S = r.standard_normal((K, V)).astype(np.float32)
+    codes, sc = formats.quantize_state_h32(S)
+    for k in range(K):
+        for g in range(V // 32):
+            c1, s1 = formats.quantize_rotated_groups(formats.hadamard32(S[k, 32 * g:32 * g + 32])[None])
+            assert s1[0] == sc[g, k] and np.array_equal(c1[0], codes[k, 32 * g:32 * g + 32])
+
+
+def pin_h32_codec_error_and_extremes():
+    """Round trip error within the rotated-domain bound (half a code step per
+    element, carried over unchanged by an orthonormal rotation); the largest
+    rotated value codes to +-127; zero groups store 0; sign symmetry; a spike
+    spreads over the whole group."""
+    r = np.random.default_rng(82)
+    K, V = 8, 64
+    S = (r.standard_normal((K, V)) * np.exp(r.uniform(-6, 6, (K, 1)))).astype(np.float32)
+    S[3, :32] = 0
+    codes, sc = formats.quantize_state_h32(S)
+    deq = formats.dequantize_state_h32(codes, sc)
+    Hs = np.array([[(-1.0) ** bin(i & j).count("1") for j in range(32)] for i in range(32)]) / math.sqrt(32)
+    for k in range(K):
+        for g in range(V // 32):
+            x = S[k, 32 * g:32 * g + 32].astype(np.float64)
+            y = Hs @ x
+            amax = np.max(np.abs(y))
+            if amax == 0:
+                assert sc[g, k] == 0 and not codes[k, 32 * g:32 * g + 32].any()
+                assert not deq[k, 32 * g:32 * g + 32].any()
+                continue
+            assert abs(sc[g, k] - amax / 127) <= 2e-6 * amax / 127
+            assert np.max(np.abs(codes[k, 32 * g:32 * g + 32].astype(int))) == 127
+            err = np.linalg.norm(deq[k, 32 * g:32 * g + 32] - x)
+            assert err <= math.sqrt(32) * 0.5 * sc[g, k] * (1 + 1e-4) + 1e-5 * np.linalg.norm(x), (k, g)
+    cn, sn = formats.quantize_state_h32(-S)
+    assert np.array_equal(sn, sc) and np.array_equal(cn, -codes)
+    spike = np.zeros((1, 32), np.float32)
+    spike[0, 7] = 3.0
+    c, s = formats.quantize_state_h32(spike)
+    assert np.all(np.abs(c.astype(int)) == 127)
+    assert np.allclose(formats.dequantize_state_h32(c, s), spike, rtol=0, atol=1e-6)
+
+
+def pin_h32_state_decode_is_codec_around_f32_step():
+    """A decode on an int8_hadamard32 pool is the fp32 decode of the decoded
+    state, with the new state stored through the codec (both layouts)."""
+    r = np.random.default_rng(83)
+    B, T, H, HV, K, V = 2, 2, 1, 2, 8, 32
+    q, k = r.standard_normal((B, T, H, K)), r.standard_normal((B, T, H, K))
+    v = r.standard_normal((B, T, HV, V))
+    a, b = r.standard_normal((B, T, HV)), r.standard_normal((B, T, HV))
+    A_log, dt = r.uniform(0, 2, HV), r.uniform(-1, 1, HV)
+    for layout in ("K_FIRST", "V_FIRST"):
+        pool8, sc8, pool32 = {}, {}, {}
+        for slot in range(2):
+            for hv in range(HV):
+                c = np.clip(np.rint(r.standard_normal((K, V)) * 40), -127, 127).astype(np.int8)
+                s = r.uniform(1e-3, 2e-3, (V // 32, K)).astype(np.float32)
+                pool8[slot, hv] = O._from_kv(c, layout)
+                sc8[slot, hv] = s
+                pool32[slot, hv] = O._from_kv(formats.dequantize_state_h32(c, s), layout)
+        idx = np.array([1, 0])
+        o8, w8 = O.gdn_decode_slots(q, k, v, a, b, A_log, dt, pool8, idx, layout=layout,
+                                    state_dtype="int8_hadamard32", state_scales=sc8)
+        o32, w32 = O.gdn_decode_slots(q[:, :1], k[:, :1], v[:, :1], a[:, :1], b[:, :1], A_log, dt, pool32, idx,
+                                      layout=layout)
+        assert np.array_equal(o8[:, :1], o32)
+        first8 = O.gdn_decode_slots(q[:, :1], k[:, :1], v[:, :1], a[:, :1], b[:, :1], A_log, dt, pool8, idx,
+                                    layout=layout, state_dtype="int8_hadamard32", state_scales=sc8)[1]
+        for key, (st32, _) in w32.items():
+            c, s = formats.quantize_state_h32(O._to_kv(st32, layout))
+            assert np.array_equal(O._to_kv(first8[key][0], layout), c) and np.array_equal(first8[key][1], s)
+        assert set(w8) == set(w32)
+
+
 ALL_PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]

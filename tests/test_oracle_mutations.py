@@ -66,6 +66,56 @@ def _e4m3_half_away(x):
 
 
 _ORIG_E4M3 = formats.e4m3_encode
+_ORIG_FWHT = formats.fwht32
+_ORIG_H32_QUANT = formats.quantize_state_h32
+_ORIG_H32_DEQUANT = formats.dequantize_state_h32
+
+
+def _fwht_wrong_sign(x):
+    """Butterfly (a + b, b - a) instead of (a + b, a - b)."""
+    y = np.array(x, copy=True)
+    lead = y.shape[:-1]
+    span = 1
+    while span < 32:
+        y = y.reshape(lead + (32 // (2 * span), 2, span))
+        a, b = y[..., 0, :].copy(), y[..., 1, :].copy()
+        y[..., 0, :] = a + b
+        y[..., 1, :] = b - a
+        y = y.reshape(lead + (32,))
+        span *= 2
+    return y
+
+
+def _h32_scales_128(amax):
+    amax = np.asarray(amax, np.float32)
+    with np.errstate(all="ignore"):
+        s = (amax / np.float32(128)).astype(np.float32)
+        r = (np.float32(1) / s).astype(np.float32)
+    zero = ~(amax > 0) | ~np.isfinite(r)
+    return np.where(zero, 0, s).astype(np.float32), np.where(zero, 0, r).astype(np.float32)
+
+
+def _int8_half_away(y):
+    y = np.asarray(y, np.float64)
+    return np.clip(np.sign(y) * np.floor(np.abs(y) + 0.5), -127, 127).astype(np.int8)
+
+
+def _h32_group_along_keys(S_kv):
+    """Groups of 32 key channels per value column instead of 32 values per key channel."""
+    S = np.asarray(S_kv, np.float32)
+    K, V = S.shape
+    if K % 32:
+        c, s = _ORIG_H32_QUANT(S)
+        return c, s[::-1].copy()
+    c, s = _ORIG_H32_QUANT(np.ascontiguousarray(S.T))
+    return c.T.copy(), s
+
+
+def _h32_dequant_unrotated(codes_kv, scales):
+    codes = np.asarray(codes_kv, np.int8)
+    K, V = codes.shape
+    sc = np.asarray(scales, np.float32).T
+    return (codes.reshape(K, V // 32, 32).astype(np.float32) * sc[..., None]).astype(np.float32).reshape(K, V)
 
 MUTATIONS = {
     "read_transposed": (O, "delta_read", lambda S, k: S @ k),
@@ -95,6 +145,12 @@ MUTATIONS = {
                        lambda x: (np.ascontiguousarray(np.asarray(x, np.float32)).view(np.uint32) >> 16).astype(np.uint16)),
     "e4m3_half_away": (formats, "e4m3_encode", _e4m3_half_away),
     "tile_scale_256": (formats, "quantize_tile", _tile_wrong_max),
+    "h32_butterfly_sign": (formats, "fwht32", _fwht_wrong_sign),
+    "h32_unnormalised": (formats, "hadamard32", lambda x: _ORIG_FWHT(np.asarray(x))),
+    "h32_scale_128": (formats, "h32_scales", _h32_scales_128),
+    "int8_half_away": (formats, "int8_round", _int8_half_away),
+    "h32_group_along_keys": (formats, "quantize_state_h32", _h32_group_along_keys),
+    "h32_decode_unrotated": (formats, "dequantize_state_h32", _h32_dequant_unrotated),
 }
 
 

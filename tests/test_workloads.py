@@ -54,6 +54,11 @@ def test_layouts_hold_same_logical_state():
     codes, scales = W.slot_state(4, 0, 2, 8, 128, "V_FIRST", "fp8_e4m3", 64)
     assert codes.dtype == np.uint8 and scales.shape == (2, 2)
     assert not np.any((codes & 0x7F) == 0x7F)   # no NaN codes
+    c8k, s8k = W.slot_state(5, 1, 2, 8, 64, "K_FIRST", "int8_hadamard32")
+    c8v, s8v = W.slot_state(5, 1, 2, 8, 64, "V_FIRST", "int8_hadamard32")
+    assert c8k.dtype == np.int8 and np.array_equal(c8k, c8v.transpose(0, 2, 1))
+    assert s8k.shape == (2, 2, 8) and np.array_equal(s8k, s8v) and np.all(s8k > 0)
+    assert int(np.abs(c8k.astype(int)).max()) <= 127
 
 
 def test_bf16_inputs_are_representable():

@@ -22,6 +22,8 @@ Workloads (sizes and distributions of the decode problems the pages pose):
 * ``fp8``   GDN slot pool, T=1, B=1024, H=16, HV=32, K=V=128, bf16 inputs,
   fp8_e4m3 pool [1024, 32, 128, 128] with one fp32 scale per [128, 64] tile,
   indices a random permutation of 1024; seed 4.
+* ``int8``  as ``fp8`` with an int8_hadamard32 pool [1024, 32, 128, 128] and
+  fp32 scales [1024, 32, 4, 128] (one per 32 values of a key channel); seed 5.
 
 Distributions (all workloads): q, k, v ~ N(0, 1); A_log ~ U(0, 2.8);
 a ~ N(0, 1); dt_bias ~ U(-1, 1); b ~ N(0, 1); initial state ~ N(0, 0.1)
@@ -53,7 +55,7 @@ class Workload:
     K: int
     V: int
     in_dtype: str             # 'f32' | 'bf16'
-    state_dtype: str          # 'f32' | 'bf16' | 'fp8_e4m3'
+    state_dtype: str          # 'f32' | 'bf16' | 'fp8_e4m3' | 'int8_hadamard32'
     layout: str               # 'K_FIRST' | 'V_FIRST'
     num_slots: int = 0        # slot pools
     page_size: int = 0        # paged pools
@@ -77,6 +79,9 @@ WORKLOADS: Dict[str, Workload] = {
     "fp8": Workload("fp8", "gdn_slots", 4, B=1024, T=1, H=16, HV=32, K=128, V=128,
                     in_dtype="bf16", state_dtype="fp8_e4m3", layout="V_FIRST",
                     num_slots=1024, block_v=64),
+    "int8": Workload("int8", "gdn_slots", 5, B=1024, T=1, H=16, HV=32, K=128, V=128,
+                     in_dtype="bf16", state_dtype="int8_hadamard32", layout="V_FIRST",
+                     num_slots=1024),
 }
 
 
@@ -252,6 +257,9 @@ def slot_state(seed, slot, HV, K, V, layout, state_dtype, block_v=64):
     fp8_e4m3: codes from torch's float8_e4m3fn cast of N(0, 1) * 100 clipped
     to +-440, with one scale ~ 1e-3 * U(0.75, 1.25) per [K, block_v] tile, so
     that decoded values are near N(0, 0.1).
+    int8_hadamard32: codes N(0, 1) * 42 rounded and clipped to +-127, with
+    one scale ~ (0.1 / 42) * U(0.75, 1.25) per (32-value group, key channel),
+    scales [HV, V / 32, K]; decoded values are again near N(0, 0.1).
     The logical [K, V] content is drawn first and then laid out, so a K_FIRST
     and a V_FIRST pool built from one seed hold the same logical states.
     """
@@ -261,6 +269,9 @@ def slot_state(seed, slot, HV, K, V, layout, state_dtype, block_v=64):
     elif state_dtype == "fp8_e4m3":
         logical = np.clip(r.standard_normal((HV, K, V), dtype=np.float32) * np.float32(100.0),
                           -440.0, 440.0)
+    elif state_dtype == "int8_hadamard32":
+        logical = np.clip(np.rint(r.standard_normal((HV, K, V), dtype=np.float32) * np.float32(42.0)),
+                          -127, 127).astype(np.int8)
     else:
         raise ValueError(state_dtype)
     stored = logical if layout == "K_FIRST" else np.ascontiguousarray(logical.transpose(0, 2, 1))
@@ -269,6 +280,9 @@ def slot_state(seed, slot, HV, K, V, layout, state_dtype, block_v=64):
     if state_dtype == "bf16":
         bits = torch.from_numpy(np.ascontiguousarray(stored)).to(torch.bfloat16).view(torch.int16)
         return bits.numpy().view(np.uint16), None
+    if state_dtype == "int8_hadamard32":
+        scales = (np.float32(0.1 / 42.0) * r.uniform(0.75, 1.25, size=(HV, V // 32, K))).astype(np.float32)
+        return np.ascontiguousarray(stored), scales
     codes = torch.from_numpy(np.ascontiguousarray(stored)).to(torch.float8_e4m3fn).view(torch.uint8)
     scales = (np.float32(1e-3) * r.uniform(0.75, 1.25, size=(HV, V // block_v))).astype(np.float32)
     return codes.numpy(), scales
@@ -288,12 +302,13 @@ def host_pool(seed, slots: Sequence[int], HV, K, V, layout, state_dtype, block_v
 
 
 def torch_state_dtype(state_dtype):
-    return {"f32": torch.float32, "bf16": torch.bfloat16, "fp8_e4m3": torch.uint8}[state_dtype]
+    return {"f32": torch.float32, "bf16": torch.bfloat16, "fp8_e4m3": torch.uint8,
+            "int8_hadamard32": torch.int8}[state_dtype]
 
 
 def device_pool(seed, num_slots, HV, K, V, layout, state_dtype, block_v=64,
                 exact_slots: Optional[Sequence[int]] = None, device="cuda"):
-    """Allocate and fill a device pool [num_slots, HV, *layout*] (+ fp8 scales).
+    """Allocate and fill a device pool [num_slots, HV, *layout*] (+ fp8 or int8 scales).
 
     Slots in ``exact_slots`` get the per-slot seeded host content of
     ``slot_state`` (what the oracle regenerates); every other slot gets the
@@ -312,6 +327,15 @@ def device_pool(seed, num_slots, HV, K, V, layout, state_dtype, block_v=64,
             x = torch.randn((s1 - s0,) + shape[1:], generator=g, device=device) * 100.0
             pool[s0:s1] = x.clamp_(-440.0, 440.0).to(torch.float8_e4m3fn).view(torch.uint8)
         scales.uniform_(0.75e-3, 1.25e-3, generator=g)
+    elif state_dtype == "int8_hadamard32":
+        pool = torch.empty(shape, dtype=torch.int8, device=device)
+        scales = torch.empty((num_slots, HV, V // 32, K), dtype=torch.float32, device=device)
+        chunk = max(1, (1 << 28) // (HV * K * V))
+        for s0 in range(0, num_slots, chunk):
+            s1 = min(num_slots, s0 + chunk)
+            x = torch.randn((s1 - s0,) + shape[1:], generator=g, device=device) * 42.0
+            pool[s0:s1] = x.round_().clamp_(-127.0, 127.0).to(torch.int8)
+        scales.uniform_(0.75 * 0.1 / 42.0, 1.25 * 0.1 / 42.0, generator=g)
     else:
         pool = torch.empty(shape, dtype=torch_state_dtype(state_dtype), device=device)
         chunk = max(1, (1 << 28) // (HV * K * V))
