@@ -14,6 +14,8 @@ Functions (same names as the C entry points):
 * ``gdn_paged_decode_slots`` (read_page, write_page) rows for a page table
 * ``kda_decode_varlen``     KDA (per-key-channel gate) varlen decode
 * ``gdn_state_quantize_fp8`` / ``gdn_state_dequantize_fp8``  fp8 tile codec
+* ``gdn_state_quantize_int8h32`` / ``gdn_state_dequantize_int8h32``
+  int8_hadamard32 codec (an int8 pool with fp32 scales [slots, HV, V/32, K])
 """
 
 from __future__ import annotations
@@ -28,7 +30,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libgdn_b200.so")
 
 GDN_OK, GDN_ERR_INVALID_ARG, GDN_ERR_UNSUPPORTED, GDN_ERR_CUDA = 0, -1, -2, -3
-GDN_F32, GDN_BF16, GDN_FP8_E4M3 = 0, 1, 2
+GDN_F32, GDN_BF16, GDN_FP8_E4M3, GDN_INT8_H32 = 0, 1, 2, 3
 GDN_I32, GDN_I64 = 0, 1
 GDN_K_FIRST, GDN_V_FIRST = 0, 1
 GDN_READOUT_WORKING, GDN_READOUT_STORED = 0, 1
@@ -118,10 +120,13 @@ def lib() -> ctypes.CDLL:
         L.gdn_paged_decode_slots.argtypes = [_vp, _vp, _vp, _i32, _i64, _i32, _i64, _i32, _vp, _vp, _vp]
         L.gdn_state_quantize_fp8.argtypes = [_vp, _vp, _vp, _i64, _i32, _i32, _i32, _i32, _vp]
         L.gdn_state_dequantize_fp8.argtypes = [_vp, _vp, _vp, _i64, _i32, _i32, _i32, _i32, _vp]
+        L.gdn_state_quantize_int8h32.argtypes = [_vp, _vp, _vp, _i64, _i32, _i32, _i32, _vp]
+        L.gdn_state_dequantize_int8h32.argtypes = [_vp, _vp, _vp, _i64, _i32, _i32, _i32, _vp]
         L.gdn_status_string.argtypes = [ctypes.c_int]
         L.gdn_status_string.restype = ctypes.c_char_p
         for f in ("gdn_decode_slots", "gdn_decode_paged", "kda_decode_varlen", "gdn_paged_decode_slots",
-                  "gdn_state_quantize_fp8", "gdn_state_dequantize_fp8", "gdn_prefill_paged"):
+                  "gdn_state_quantize_fp8", "gdn_state_dequantize_fp8", "gdn_prefill_paged",
+                  "gdn_state_quantize_int8h32", "gdn_state_dequantize_int8h32"):
             getattr(L, f).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -160,6 +165,8 @@ def _state_dtype(t: torch.Tensor) -> int:
         return GDN_BF16
     if t.dtype in (torch.uint8, torch.float8_e4m3fn):
         return GDN_FP8_E4M3
+    if t.dtype == torch.int8:
+        return GDN_INT8_H32
     raise ValueError(f"unsupported state dtype {t.dtype}")
 
 
@@ -194,7 +201,13 @@ def _pool(state_pool, state_scales, layout, block_v, K, V, HV) -> gdn_state_pool
             raise ValueError("an fp8 state pool needs fp32 state_scales [slots, HV, V/block_v]")
         if tuple(state_scales.shape) != (state_pool.shape[0], HV, V // block_v):
             raise ValueError("state_scales must be [slots, HV, V/block_v]")
-    return gdn_state_pool(_ptr(state_pool), _ptr(state_scales) if sdt == GDN_FP8_E4M3 else None,
+    if sdt == GDN_INT8_H32:
+        if state_scales is None or state_scales.dtype != torch.float32:
+            raise ValueError("an int8_hadamard32 state pool needs fp32 state_scales [slots, HV, V/32, K]")
+        if tuple(state_scales.shape) != (state_pool.shape[0], HV, V // 32, K):
+            raise ValueError("state_scales must be [slots, HV, V/32, K]")
+    coded = sdt in (GDN_FP8_E4M3, GDN_INT8_H32)
+    return gdn_state_pool(_ptr(state_pool), _ptr(state_scales) if coded else None,
                           state_pool.shape[0], sdt, lay, block_v, 0)
 
 
@@ -454,6 +467,31 @@ def gdn_state_dequantize_fp8(codes, scales, *, block_v=64, layout="V_FIRST", out
     return out
 
 
+def gdn_state_quantize_int8h32(src, *, layout="V_FIRST", codes=None,
+                               scales=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """fp32 states [N, K, V] (K_FIRST) or [N, V, K] (V_FIRST) -> (int8 codes, scales [N, V/32, K])."""
+    N = src.shape[0]
+    lay = _LAYOUTS[layout]
+    K, V = (src.shape[1], src.shape[2]) if lay == GDN_K_FIRST else (src.shape[2], src.shape[1])
+    codes = _out(codes, tuple(src.shape), torch.int8, src)
+    scales = _out(scales, (N, V // 32, K), torch.float32, src)
+    _check(lib().gdn_state_quantize_int8h32(_ptr(src), _ptr(codes), _ptr(scales), N, K, V, lay, _stream(src)),
+           "gdn_state_quantize_int8h32")
+    return codes, scales
+
+
+def gdn_state_dequantize_int8h32(codes, scales, *, layout="V_FIRST", out=None) -> torch.Tensor:
+    N = codes.shape[0]
+    lay = _LAYOUTS[layout]
+    K, V = (codes.shape[1], codes.shape[2]) if lay == GDN_K_FIRST else (codes.shape[2], codes.shape[1])
+    _expect(scales, (N, V // 32, K), "scales")
+    out = _out(out, tuple(codes.shape), torch.float32, codes)
+    _check(lib().gdn_state_dequantize_int8h32(_ptr(codes), _ptr(scales), _ptr(out), N, K, V, lay, _stream(codes)),
+           "gdn_state_dequantize_int8h32")
+    return out
+
+
 __all__ = ["gdn_decode_slots", "gdn_decode_paged", "gdn_prefill_paged", "gdn_paged_decode_slots", "kda_decode_varlen",
-           "gdn_state_quantize_fp8", "gdn_state_dequantize_fp8", "gdn_status_string", "GDNError",
+           "gdn_state_quantize_fp8", "gdn_state_dequantize_fp8", "gdn_state_quantize_int8h32",
+           "gdn_state_dequantize_int8h32", "gdn_status_string", "GDNError",
            "LIB_PATH", "lib"]

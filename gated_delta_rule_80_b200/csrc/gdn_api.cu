@@ -1,5 +1,6 @@
 // C ABI of the decode library: host-side validation, launch selection and
-// the small auxiliary kernels (paged slot rows, fp8 tile codec).
+// the small auxiliary kernels (paged slot rows, fp8 tile codec,
+// int8_hadamard32 codec).
 //
 // Validation runs before any CUDA call, so a rejected call touches neither
 // the device nor the stream. The device is taken from the state pool's
@@ -35,7 +36,7 @@ bool ptrs_ok(std::initializer_list<const void*> vec16, std::initializer_list<std
 }
 bool head_dim_ok(int x) { return x == 32 || x == 64 || x == 128 || x == 256; }
 bool io_dtype_ok(int d) { return d == GDN_F32 || d == GDN_BF16; }
-bool state_dtype_ok(int d) { return d == GDN_F32 || d == GDN_BF16 || d == GDN_FP8_E4M3; }
+bool state_dtype_ok(int d) { return d == GDN_F32 || d == GDN_BF16 || d == GDN_FP8_E4M3 || d == GDN_INT8_H32; }
 bool layout_ok(int l) { return l == GDN_K_FIRST || l == GDN_V_FIRST; }
 
 // Checks of a state pool shared by every entry point.
@@ -48,6 +49,10 @@ int check_pool(const gdn_state_pool& pool, int V) {
     const int bv = pool.block_v == 0 ? 64 : pool.block_v;
     if (bv <= 0 || V % bv != 0) return GDN_ERR_INVALID_ARG;
     if (bv != 64) return GDN_ERR_UNSUPPORTED;
+  }
+  if (pool.dtype == GDN_INT8_H32) {
+    if (pool.scales == nullptr || !aligned16(pool.scales)) return GDN_ERR_INVALID_ARG;
+    if (V % 64 != 0) return GDN_ERR_UNSUPPORTED;  // the kernels' tile is two scale groups
   }
   return GDN_OK;
 }
@@ -99,19 +104,20 @@ template <int L, int SDT, int K, int GATE, int IDX>
 int launch_one(StepParams p, int B, cudaStream_t s) {
   p.G = p.HV / p.H;
   if (B > 65535) return GDN_ERR_INVALID_ARG;  // grid z
-  if constexpr (L == L_VFIRST && GATE == GATE_SCALAR) {
+  constexpr bool CODED = (SDT == ST_FP8 || SDT == ST_I8H);
+  if constexpr (L == L_VFIRST && GATE == GATE_SCALAR && SDT != ST_I8H) {
     if (p.T == 1) return launch_tile1<SDT, K, IDX>(p, B, s);
   }
   if constexpr (L == L_KFIRST) {
     constexpr int VTW = (K == 256) ? 8 : 16;  // columns per warp
-    if constexpr (SDT == ST_FP8) {
-      return launch_seq_nw<L, SDT, K, GATE, IDX, 64 / VTW>(p, B, s);  // the 64-column scale tile
+    if constexpr (CODED) {
+      return launch_seq_nw<L, SDT, K, GATE, IDX, 64 / VTW>(p, B, s);  // 64-column tiles of scale groups
     } else {
       if (p.V % (4 * VTW) != 0) return launch_seq_nw<L, SDT, K, GATE, IDX, 2>(p, B, s);
       return launch_seq_nw<L, SDT, K, GATE, IDX, 4>(p, B, s);
     }
   } else {
-    return launch_seq_nw<L, SDT, K, GATE, IDX, (SDT == ST_FP8 && K == 256) ? 8 : 4>(p, B, s);
+    return launch_seq_nw<L, SDT, K, GATE, IDX, (CODED && K == 256) ? 8 : 4>(p, B, s);
   }
 }
 
@@ -132,6 +138,7 @@ int launch_sdt(const StepParams& p, int sdt, int K, int B, cudaStream_t s) {
     case GDN_F32: return launch_k<L, ST_F32, GATE, IDX>(p, K, B, s);
     case GDN_BF16: return launch_k<L, ST_BF16, GATE, IDX>(p, K, B, s);
     case GDN_FP8_E4M3: return launch_k<L, ST_FP8, GATE, IDX>(p, K, B, s);
+    case GDN_INT8_H32: return launch_k<L, ST_I8H, GATE, IDX>(p, K, B, s);
     default: return GDN_ERR_INVALID_ARG;
   }
 }
@@ -247,6 +254,110 @@ int launch_quantize(const float* src, uint8_t* codes, float* scales, int64_t n, 
     default: return GDN_ERR_INVALID_ARG;
   }
   return launch_status();
+}
+
+// int8_hadamard32 codec: one thread per (state, 32-value group, key
+// channel), consecutive threads on consecutive key channels. The 32 values
+// are rotated in registers by the butterfly order of fwht32_regs, scaled by
+// the binary32 nearest 1/sqrt(32), and coded against amax / 127.
+template <int LAYOUT>
+__global__ void __launch_bounds__(128) h32_quantize_kernel(const float* src, int8_t* codes, float* scales, int K,
+                                                           int V, int64_t n_items) {
+  const int64_t it = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (it >= n_items) return;
+  const int G = V / 32;
+  const int k = static_cast<int>(it % K);
+  const int64_t ng = it / K;
+  const int g = static_cast<int>(ng % G);
+  const int64_t base = (ng / G) * (int64_t)K * V;
+  float x[32];
+  if constexpr (LAYOUT == L_VFIRST) {
+#pragma unroll
+    for (int j = 0; j < 32; ++j) x[j] = src[base + (int64_t)(32 * g + j) * K + k];
+  } else {
+    const float4* p4 = reinterpret_cast<const float4*>(src + base + (int64_t)k * V + 32 * g);
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      const float4 f = p4[c];
+      x[4 * c] = f.x; x[4 * c + 1] = f.y; x[4 * c + 2] = f.z; x[4 * c + 3] = f.w;
+    }
+  }
+  fwht32_regs(x);
+  float m = 0.f;
+#pragma unroll
+  for (int j = 0; j < 32; ++j) {
+    x[j] = __fmul_rn(x[j], inv_sqrt32());
+    m = absmax_acc(m, x[j]);
+  }
+  float s, r;
+  h32_scale_of(fabsf(m), s, r);
+  uint32_t w[8];
+#pragma unroll
+  for (int c = 0; c < 8; ++c) {
+    float y[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) y[e] = fminf(fmaxf(__fmul_rn(x[4 * c + e], r), -kInt8Max), kInt8Max);
+    w[c] = float_to_i8x4(y[0], y[1], y[2], y[3]);
+  }
+  if constexpr (LAYOUT == L_VFIRST) {
+#pragma unroll
+    for (int j = 0; j < 32; ++j)
+      codes[base + (int64_t)(32 * g + j) * K + k] = static_cast<int8_t>((w[j / 4] >> (8 * (j % 4))) & 0xffu);
+  } else {
+    uint4* c4 = reinterpret_cast<uint4*>(codes + base + (int64_t)k * V + 32 * g);
+    c4[0] = make_uint4(w[0], w[1], w[2], w[3]);
+    c4[1] = make_uint4(w[4], w[5], w[6], w[7]);
+  }
+  scales[ng * K + k] = s;
+}
+
+template <int LAYOUT>
+__global__ void __launch_bounds__(128) h32_dequantize_kernel(const int8_t* codes, const float* scales, float* dst,
+                                                             int K, int V, int64_t n_items) {
+  const int64_t it = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (it >= n_items) return;
+  const int G = V / 32;
+  const int k = static_cast<int>(it % K);
+  const int64_t ng = it / K;
+  const int g = static_cast<int>(ng % G);
+  const int64_t base = (ng / G) * (int64_t)K * V;
+  const float s = scales[ng * K + k];
+  float x[32];
+  if constexpr (LAYOUT == L_VFIRST) {
+#pragma unroll
+    for (int j = 0; j < 32; ++j) x[j] = static_cast<float>(codes[base + (int64_t)(32 * g + j) * K + k]);
+  } else {
+    const uint4* c4 = reinterpret_cast<const uint4*>(codes + base + (int64_t)k * V + 32 * g);
+    const uint4 a = c4[0], b = c4[1];
+    const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+#pragma unroll
+    for (int c = 0; c < 8; ++c) i8x4_to_float(w[c], x + 4 * c);
+  }
+#pragma unroll
+  for (int j = 0; j < 32; ++j) x[j] = __fmul_rn(x[j], s);
+  fwht32_regs(x);
+#pragma unroll
+  for (int j = 0; j < 32; ++j) x[j] = __fmul_rn(x[j], inv_sqrt32());
+  if constexpr (LAYOUT == L_VFIRST) {
+#pragma unroll
+    for (int j = 0; j < 32; ++j) dst[base + (int64_t)(32 * g + j) * K + k] = x[j];
+  } else {
+    float4* d4 = reinterpret_cast<float4*>(dst + base + (int64_t)k * V + 32 * g);
+#pragma unroll
+    for (int c = 0; c < 8; ++c) d4[c] = make_float4(x[4 * c], x[4 * c + 1], x[4 * c + 2], x[4 * c + 3]);
+  }
+}
+
+// Shared checks of the two int8_hadamard32 codec calls; n_items out = threads.
+int h32_codec_args(const void* a, const void* b, const void* c, int64_t n_states, int K, int V, int layout,
+                   int64_t& n_items) {
+  if (n_states < 0 || !head_dim_ok(K) || !head_dim_ok(V) || !layout_ok(layout)) return GDN_ERR_INVALID_ARG;
+  n_items = n_states * (V / 32) * K;
+  if (n_states == 0) return GDN_OK;
+  if (a == nullptr || b == nullptr || c == nullptr) return GDN_ERR_INVALID_ARG;
+  if (!aligned16(a) || !aligned16(b) || !aligned16(c)) return GDN_ERR_INVALID_ARG;
+  if ((n_items + 127) / 128 > INT_MAX) return GDN_ERR_INVALID_ARG;
+  return GDN_OK;
 }
 
 }  // namespace
@@ -457,6 +568,32 @@ int gdn_state_dequantize_fp8(const uint8_t* codes, const float* scales, float* d
     fp8_dequantize_kernel<L_VFIRST><<<static_cast<unsigned>(blocks), threads, 0, s>>>(codes, scales, dst, n_chunks, K, V);
   else
     fp8_dequantize_kernel<L_KFIRST><<<static_cast<unsigned>(blocks), threads, 0, s>>>(codes, scales, dst, n_chunks, K, V);
+  return launch_status();
+}
+
+int gdn_state_quantize_int8h32(const float* src, int8_t* codes, float* scales, int64_t n_states, int32_t K,
+                               int32_t V, int32_t layout, gdn_stream_t stream) {
+  int64_t n = 0;
+  if (const int rc = h32_codec_args(src, codes, scales, n_states, K, V, layout, n)) return rc;
+  if (n_states == 0) return GDN_OK;
+  if (const int rc = select_device(src)) return rc;
+  const unsigned blocks = static_cast<unsigned>((n + 127) / 128);
+  const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (layout == GDN_V_FIRST) h32_quantize_kernel<L_VFIRST><<<blocks, 128, 0, s>>>(src, codes, scales, K, V, n);
+  else h32_quantize_kernel<L_KFIRST><<<blocks, 128, 0, s>>>(src, codes, scales, K, V, n);
+  return launch_status();
+}
+
+int gdn_state_dequantize_int8h32(const int8_t* codes, const float* scales, float* dst, int64_t n_states, int32_t K,
+                                 int32_t V, int32_t layout, gdn_stream_t stream) {
+  int64_t n = 0;
+  if (const int rc = h32_codec_args(codes, scales, dst, n_states, K, V, layout, n)) return rc;
+  if (n_states == 0) return GDN_OK;
+  if (const int rc = select_device(dst)) return rc;
+  const unsigned blocks = static_cast<unsigned>((n + 127) / 128);
+  const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (layout == GDN_V_FIRST) h32_dequantize_kernel<L_VFIRST><<<blocks, 128, 0, s>>>(codes, scales, dst, K, V, n);
+  else h32_dequantize_kernel<L_KFIRST><<<blocks, 128, 0, s>>>(codes, scales, dst, K, V, n);
   return launch_status();
 }
 

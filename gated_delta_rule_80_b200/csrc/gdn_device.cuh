@@ -13,7 +13,7 @@ namespace gdn {
 // ---------------------------------------------------------------------------
 // enums shared with the host side (values match include/gdn.h)
 // ---------------------------------------------------------------------------
-enum StateFmt : int { ST_F32 = 0, ST_BF16 = 1, ST_FP8 = 2 };
+enum StateFmt : int { ST_F32 = 0, ST_BF16 = 1, ST_FP8 = 2, ST_I8H = 3 };
 enum Layout : int { L_KFIRST = 0, L_VFIRST = 1 };
 enum IndexMode : int { IDX_SLOTS = 0, IDX_PAGED = 1 };
 enum GateKind : int { GATE_SCALAR = 0, GATE_VECTOR = 1 };
@@ -48,7 +48,7 @@ struct StepParams {
   const float* A_log;   // [HV]
   const float* dt_bias; // GDN [HV]; KDA [HV, K]
   void* pool;           // [num_slots, HV, state]
-  float* scales;        // fp8: [num_slots, HV, V / 64]
+  float* scales;        // fp8: [num_slots, HV, V / 64]; int8: [num_slots, HV, V / 32, K]
   const void* idx;      // slots: state_indices [B]; paged: page_indices [nnz]
   const void* indptr;   // paged: page_indptr [B+1]; varlen: cu_seqlens [B+1] int32
   const void* lastlen;  // paged: last_page_len [B]
@@ -74,6 +74,7 @@ template <int SDT> struct StateTraits;
 template <> struct StateTraits<ST_F32> { static constexpr int EPL = 4, BYTES = 4; };
 template <> struct StateTraits<ST_BF16> { static constexpr int EPL = 8, BYTES = 2; };
 template <> struct StateTraits<ST_FP8> { static constexpr int EPL = 16, BYTES = 1; };
+template <> struct StateTraits<ST_I8H> { static constexpr int EPL = 16, BYTES = 1; };
 
 // Streaming 16-byte load/store: the state is touched once per launch, so it
 // should not displace anything in L1/L2 ("evict first").
@@ -107,7 +108,83 @@ __device__ __forceinline__ uint16_t float2_to_e4m3x2(float x, float y) {
   return static_cast<uint16_t>(__nv_cvt_float2_to_fp8x2(make_float2(x, y), __NV_SATFINITE, __NV_E4M3));
 }
 
-// Decode 16 stored bytes into EPL floats (fp8 codes are returned unscaled).
+// ---------------------------------------------------------------------------
+// int8_hadamard32 codes: each (key channel, 32 values) group of the state is
+// held rotated by R = H32 / sqrt(32) (Sylvester order), as int8 codes with one
+// fp32 scale s = amax / 127 per group.
+// ---------------------------------------------------------------------------
+constexpr float kInt8Max = 127.0f;
+// 1.5 * 2^23: adding it to |x| < 2^22 rounds x to an integer (ties to even)
+// and leaves that integer in the low mantissa bits, two's complement.
+constexpr float kRoundMagic = 12582912.0f;
+// 2^23 + 128: a byte b placed under the exponent of 2^23 reads 2^23 + b.
+constexpr float kByteBias = 8388736.0f;
+
+// The binary32 nearest to 1/sqrt(32) (a quarter of the one nearest 1/sqrt(2)).
+__device__ __forceinline__ float inv_sqrt32() { return __uint_as_float(0x3E3504F3u); }
+
+// 4 int8 codes (one word, low byte first) -> their values as floats, exactly:
+// flipping the sign bit of a byte gives code + 128.
+__device__ __forceinline__ void i8x4_to_float(uint32_t w, float* x) {
+  const uint32_t u = w ^ 0x80808080u;
+  const float2 bias = make_float2(-kByteBias, -kByteBias);
+  const float2 lo = __fadd2_rn(make_float2(__uint_as_float(__byte_perm(u, 0x4B000000u, 0x7540)),
+                                           __uint_as_float(__byte_perm(u, 0x4B000000u, 0x7541))), bias);
+  const float2 hi = __fadd2_rn(make_float2(__uint_as_float(__byte_perm(u, 0x4B000000u, 0x7542)),
+                                           __uint_as_float(__byte_perm(u, 0x4B000000u, 0x7543))), bias);
+  x[0] = lo.x; x[1] = lo.y; x[2] = hi.x; x[3] = hi.y;
+}
+
+// 4 floats already multiplied by the group's r (|x| <= 127.5 for finite
+// states) -> 4 int8 codes, nearest integer with ties to even.
+__device__ __forceinline__ uint32_t float_to_i8x4(float a, float b, float c, float d) {
+  const float2 m = make_float2(kRoundMagic, kRoundMagic);
+  const float2 ab = __fadd2_rn(make_float2(a, b), m);
+  const float2 cd = __fadd2_rn(make_float2(c, d), m);
+  const uint32_t lo = __byte_perm(__float_as_uint(ab.x), __float_as_uint(ab.y), 0x0040);
+  const uint32_t hi = __byte_perm(__float_as_uint(cd.x), __float_as_uint(cd.y), 0x0040);
+  return __byte_perm(lo, hi, 0x5410);
+}
+
+// Group scale from the group's amax: s = amax / 127 and r = 1 / s, both
+// correctly rounded; a zero group (or one whose r overflows) stores s = 0
+// and codes 0 (signalled by r = 0).
+__device__ __forceinline__ void h32_scale_of(float amax, float& s, float& r) {
+  s = __fdiv_rn(amax, kInt8Max);
+  r = __frcp_rn(s);
+  if (!(amax > 0.0f) || isinf(r)) { s = 0.0f; r = 0.0f; }
+}
+
+// Unnormalised 32-point Walsh-Hadamard transform of one value per lane
+// (lane = position in the group): butterflies of span 1, 2, 4, 8, 16.
+__device__ __forceinline__ float fwht_lanes(float x, int lane) {
+#pragma unroll
+  for (int span = 1; span < 32; span <<= 1) {
+    const float p = __shfl_xor_sync(kFull, x, span);
+    x = (lane & span) ? __fsub_rn(p, x) : __fadd_rn(x, p);
+  }
+  return x;
+}
+
+// The same transform of 32 values held by one thread, in the same stage
+// order: stage `span` turns the pair at (i, i + span), i & span == 0, into
+// (a + b, a - b).
+__device__ __forceinline__ void fwht32_regs(float* x) {
+#pragma unroll
+  for (int span = 1; span < 32; span <<= 1) {
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      if ((i & span) == 0) {
+        const float a = x[i], b = x[i + span];
+        x[i] = __fadd_rn(a, b);
+        x[i + span] = __fsub_rn(a, b);
+      }
+    }
+  }
+}
+
+// Decode 16 stored bytes into EPL floats (fp8 and int8 codes are returned
+// unscaled).
 template <int SDT>
 __device__ __forceinline__ void decode16(uint4 raw, float* x) {
   const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
@@ -117,6 +194,9 @@ __device__ __forceinline__ void decode16(uint4 raw, float* x) {
   } else if constexpr (SDT == ST_BF16) {
 #pragma unroll
     for (int i = 0; i < 4; ++i) { x[2 * i] = bf16_lo(w[i]); x[2 * i + 1] = bf16_hi(w[i]); }
+  } else if constexpr (SDT == ST_I8H) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) i8x4_to_float(w[i], x + 4 * i);
   } else {
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
@@ -127,7 +207,8 @@ __device__ __forceinline__ void decode16(uint4 raw, float* x) {
   }
 }
 
-// Encode EPL floats into 16 stored bytes. For fp8 the caller passes x * r.
+// Encode EPL floats into 16 stored bytes. For fp8 and int8 the caller passes
+// x * r.
 template <int SDT>
 __device__ __forceinline__ uint4 encode16(const float* x) {
   uint32_t w[4];
@@ -137,6 +218,9 @@ __device__ __forceinline__ uint4 encode16(const float* x) {
   } else if constexpr (SDT == ST_BF16) {
 #pragma unroll
     for (int i = 0; i < 4; ++i) w[i] = pack_bf16x2(x[2 * i], x[2 * i + 1]);
+  } else if constexpr (SDT == ST_I8H) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) w[i] = float_to_i8x4(x[4 * i], x[4 * i + 1], x[4 * i + 2], x[4 * i + 3]);
   } else {
 #pragma unroll
     for (int i = 0; i < 4; ++i) {

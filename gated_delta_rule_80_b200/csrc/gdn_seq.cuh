@@ -13,7 +13,7 @@
 // (for GDN alpha is a scalar and multiplies the reduced sums instead).
 //
 // Thread mappings (reductions stay inside a warp; fp8 takes one CTA barrier
-// per token for the tile amax):
+// per token for the tile amax, int8_hadamard32 two for its group scales):
 //  * V_FIRST (tile = VC stored rows of K): LPR lanes hold one row in 16-byte
 //    vectors, a thread holds NR rows; the 2 NR row sums are finished by a
 //    reduce-scatter over the row's lanes.
@@ -21,6 +21,13 @@
 //    rows; lanes are 8 row groups x 4 column quads (4 elements per lane), a
 //    thread holds K/8 rows. The 8 column sums (k and q for 4 columns) are
 //    finished by a reduce-scatter over the 8 row groups.
+//
+// int8_hadamard32 states are worked on in their rotated basis: with
+// R = H32 / sqrt(32) acting on each 32-value group (symmetric, R R = I), the
+// step commutes with the rotation -- S R advanced by R v gives S' R and reads
+// out R o -- so the tile decodes to S R directly (code * scale), the token's
+// v slice is rotated once in the prologue, the outputs are rotated back once
+// per chunk, and the state itself is never transformed.
 #pragma once
 
 #include "gdn_tile1.cuh"
@@ -51,14 +58,18 @@ struct ReduceScatterS {
 
 template <int SDT, int LAYOUT, int K, int NW>
 struct SeqShape {
-  static constexpr int TC = 8;  // tokens per prologue chunk
+  // tokens per prologue chunk (4 for int8 K=256, whose scale-group buffers
+  // would otherwise push the static shared memory past 48 KiB)
+  static constexpr int TC = (SDT == ST_I8H && K == 256) ? 4 : 8;
   // V_FIRST: 16-byte vectors (32 for a K=256 fp32 row, so that it fits a warp)
   static constexpr int VB_V = (SDT == ST_F32 && K == 256) ? 32 : 16;
   // K_FIRST: 4 elements per lane, CPL lanes per row segment (16 columns per
   // warp; 8 for K = 256 so that a thread holds K/16 rows)
   static constexpr int CPL = (K == 256) ? 2 : 4;
   static constexpr int EPL = (LAYOUT == L_VFIRST) ? VB_V / StateTraits<SDT>::BYTES : 4;
-  static constexpr int VC = (LAYOUT == L_VFIRST) ? ((SDT == ST_FP8) ? 64 : (K == 256 ? 16 : 32)) : CPL * 4 * NW;
+  // fp8: the [K, 64] scale tile; int8_hadamard32: two 32-value scale groups
+  static constexpr int VC = (LAYOUT == L_VFIRST) ? ((SDT == ST_FP8 || SDT == ST_I8H) ? 64 : (K == 256 ? 16 : 32))
+                                                 : CPL * 4 * NW;
 };
 
 template <int SDT, int LAYOUT, int K, int GATE, int IDX, int NW>
@@ -85,7 +96,14 @@ step_seq(const StepParams p) {
   static_assert(VF || NV <= RG, "one finished sum per lane");
   constexpr int REP = VF ? LPR / NV : 1;
   constexpr int KPL = K / 32;
-  constexpr int VPL = (VC + 31) / 32;
+  constexpr bool I8 = (SDT == ST_I8H);
+  // int8_hadamard32: 32-value scale groups in the tile, and partial maxima
+  // per (group, key channel): V_FIRST one per stored row a thread holds of
+  // the group, K_FIRST one per 4-column lane vector
+  constexpr int NG = I8 ? VC / 32 : 1;
+  constexpr int NP = I8 ? (VF ? 32 / NR : 8) : 1;
+  static_assert(!I8 || VC % 32 == 0, "whole scale groups per tile");
+  static_assert(!I8 || !VF || 32 % (NR * RPW) == 0, "a warp's rows stay inside one scale group");
 
   __shared__ __align__(16) float s_q[TC][K];
   __shared__ __align__(16) float s_k[TC][K];
@@ -93,6 +111,10 @@ step_seq(const StepParams p) {
   __shared__ __align__(16) float s_v[TC][VC];
   __shared__ float s_b[TC], s_qk[TC];
   __shared__ float s_amax[2][NW];
+  __shared__ __align__(16) float s_part[NG][NP][I8 ? K : 1];
+  __shared__ __align__(16) float s_sc[NG][I8 ? K : 1];
+  __shared__ __align__(16) float s_rc[NG][I8 ? K : 1];
+  __shared__ float s_ot[I8 ? TC : 1][I8 ? VC : 1];
 
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
@@ -122,6 +144,11 @@ step_seq(const StepParams p) {
   const int mycol = vidx >> 1;  // V_FIRST: row of the thread; K_FIRST: column in the lane's 4
   const int grp = VF ? lane - li : li;
   const bool writer = VF ? (!holds_q && (li % REP) == 0) : (!holds_q && (CPL == 4 || (lane & 2) == 0));
+  // int8_hadamard32: the thread's scale group in the tile, and which partial
+  // maximum of that group it writes
+  [[maybe_unused]] const int tg = VF ? (warp * NR * RPW) / 32 : c0 / 32;
+  [[maybe_unused]] const int pid =
+      VF ? lane / LPR + RPW * (((warp * NR * RPW) % 32) / (NR * RPW)) : (c0 % 32) / 4;
 
   const Unit u = resolve_unit<IDX>(p, b);
   if (threadIdx.x == 0) raise_err(p.err, u.err);
@@ -155,15 +182,19 @@ step_seq(const StepParams p) {
     for (int jj = 0; jj < NR; ++jj) raw[jj] = SV::load(src + vec_off(jj) * ST::BYTES);
 #pragma unroll
     for (int jj = 0; jj < NR; ++jj) SV::decode(raw[jj], S[jj]);
-  } else {  // 4 fp8 codes
+  } else {  // 4 fp8 or int8 codes
     uint32_t raw[NR];
 #pragma unroll
     for (int jj = 0; jj < NR; ++jj) raw[jj] = __ldcs(reinterpret_cast<const unsigned int*>(src + vec_off(jj)));
 #pragma unroll
     for (int jj = 0; jj < NR; ++jj) {
-      const float2 a = e4m3x2_to_float2(static_cast<uint16_t>(raw[jj] & 0xffffu));
-      const float2 c = e4m3x2_to_float2(static_cast<uint16_t>(raw[jj] >> 16));
-      S[jj][0] = a.x; S[jj][1] = a.y; S[jj][2] = c.x; S[jj][3] = c.y;
+      if constexpr (I8) {
+        i8x4_to_float(raw[jj], S[jj]);
+      } else {
+        const float2 a = e4m3x2_to_float2(static_cast<uint16_t>(raw[jj] & 0xffffu));
+        const float2 c = e4m3x2_to_float2(static_cast<uint16_t>(raw[jj] >> 16));
+        S[jj][0] = a.x; S[jj][1] = a.y; S[jj][2] = c.x; S[jj][3] = c.y;
+      }
     }
   }
   const int n_scale = p.V / 64;
@@ -174,6 +205,31 @@ step_seq(const StepParams p) {
     for (int jj = 0; jj < NR; ++jj)
 #pragma unroll
       for (int e = 0; e < EPL; ++e) S[jj][e] = __fmul_rn(S[jj][e], sc);
+  } else if constexpr (I8) {
+    // code * scale of the element's (group, key channel): the state in the
+    // rotated basis
+    if (!u.fresh) {
+      const float* sc = p.scales + ((u.src * p.HV + hv) * (int64_t)(V / 32) + v0 / 32 + tg) * K;
+      if constexpr (VF) {
+        float sv[EPL];
+#pragma unroll
+        for (int c = 0; c < EPL / 4; ++c) {
+          const float4 f = reinterpret_cast<const float4*>(sc + kofs)[c];
+          sv[4 * c] = f.x; sv[4 * c + 1] = f.y; sv[4 * c + 2] = f.z; sv[4 * c + 3] = f.w;
+        }
+#pragma unroll
+        for (int jj = 0; jj < NR; ++jj)
+#pragma unroll
+          for (int e = 0; e < EPL; ++e) S[jj][e] = __fmul_rn(S[jj][e], sv[e]);
+      } else {
+#pragma unroll
+        for (int jj = 0; jj < NR; ++jj) {
+          const float sj = sc[g + RG * jj];
+#pragma unroll
+          for (int e = 0; e < EPL; ++e) S[jj][e] = __fmul_rn(S[jj][e], sj);
+        }
+      }
+    }
   }
 
   const float expA = expf(p.A_log[hv]);
@@ -183,7 +239,7 @@ step_seq(const StepParams p) {
   // store the tile (in its storage format) to pool slot/page `slot`
   auto store_tile = [&](int64_t slot) {
     char* dst = reinterpret_cast<char*>(p.pool) + (slot * p.HV + hv) * head_bytes;
-    if constexpr (SDT == ST_FP8) {
+    if constexpr (SDT == ST_FP8 || I8) {
 #pragma unroll
       for (int jj = 0; jj < NR; ++jj) {
         char* a = dst + vec_off(jj);
@@ -191,7 +247,13 @@ step_seq(const StepParams p) {
         else if constexpr (EPL == 8) __stcs(reinterpret_cast<uint2*>(a), make_uint2(codes[jj][0], codes[jj][1]));
         else __stcs(reinterpret_cast<unsigned int*>(a), codes[jj][0]);
       }
-      if (threadIdx.x == 0) p.scales[(slot * p.HV + hv) * n_scale + stile] = s_last;
+      if constexpr (I8) {
+        // the tile's groups are consecutive rows of the [V/32, K] scale array
+        float* dsc = p.scales + ((slot * p.HV + hv) * (int64_t)(V / 32) + v0 / 32) * K;
+        for (int i = threadIdx.x; i < NG * K; i += NW * 32) dsc[i] = s_sc[i / K][i % K];
+      } else if (threadIdx.x == 0) {
+        p.scales[(slot * p.HV + hv) * n_scale + stile] = s_last;
+      }
     } else {
 #pragma unroll
       for (int jj = 0; jj < NR; ++jj) SV::store(dst + vec_off(jj) * ST::BYTES, SV::encode(S[jj]));
@@ -234,7 +296,11 @@ step_seq(const StepParams p) {
 #pragma unroll
         for (int e = 0; e < KPL; ++e) s_a[tt][lane * KPL + e] = decay_of(expA, gv[e] + db[e]);
       }
-      for (int c = lane; c < VC; c += 32) s_v[tt][c] = ld_in1(p.v, ((int64_t)tok * p.HV + hv) * V + v0 + c, in_bf16);
+      for (int c = lane; c < VC; c += 32) {
+        float x = ld_in1(p.v, ((int64_t)tok * p.HV + hv) * V + v0 + c, in_bf16);
+        if constexpr (I8) x = __fmul_rn(fwht_lanes(x, lane), inv_sqrt32());  // R v of one group
+        s_v[tt][c] = x;
+      }
       if (lane == 0) {
         const float braw = ld_in1(p.beta, (int64_t)tok * p.HV + hv, in_bf16);
         s_b[tt] = (p.flags & F_BETA_PROB) ? braw : sigmoid_f(braw);
@@ -406,6 +472,69 @@ step_seq(const StepParams p) {
             }
           }
         }
+      } else if constexpr (I8) {
+        // group maxima: the thread's part, then the CTA's
+        if constexpr (VF) {
+          float m[EPL];
+#pragma unroll
+          for (int e = 0; e < EPL; ++e) {
+            float a = 0.f;
+#pragma unroll
+            for (int jj = 0; jj < NR; ++jj) a = absmax_acc(a, S[jj][e]);
+            m[e] = fabsf(a);
+          }
+          float4* dp = reinterpret_cast<float4*>(&s_part[tg][pid][kofs]);
+#pragma unroll
+          for (int c = 0; c < EPL / 4; ++c) dp[c] = make_float4(m[4 * c], m[4 * c + 1], m[4 * c + 2], m[4 * c + 3]);
+        } else {
+#pragma unroll
+          for (int jj = 0; jj < NR; ++jj) {
+            float a = 0.f;
+#pragma unroll
+            for (int e = 0; e < EPL; ++e) a = absmax_acc(a, S[jj][e]);
+            s_part[tg][pid][g + RG * jj] = fabsf(a);
+          }
+        }
+        __syncthreads();
+        for (int i = threadIdx.x; i < NG * K; i += NW * 32) {
+          const int gi = i / K, kk = i % K;
+          float a = s_part[gi][0][kk];
+#pragma unroll
+          for (int pp = 1; pp < NP; ++pp) a = fmaxf(a, s_part[gi][pp][kk]);
+          float sn, r;
+          h32_scale_of(a, sn, r);
+          s_sc[gi][kk] = sn;
+          s_rc[gi][kk] = r;
+        }
+        __syncthreads();
+        // codes, and the stored state back (code * scale) where it is used again
+        const bool keep = !last || stored_readout;
+#pragma unroll
+        for (int jj = 0; jj < NR; ++jj) {
+#pragma unroll
+          for (int w4 = 0; w4 < EPL / 4; ++w4) {
+            float r4[4], s4[4];
+            if constexpr (VF) {
+              const float4 rv = *reinterpret_cast<const float4*>(&s_rc[tg][kofs + 4 * w4]);
+              const float4 sv = *reinterpret_cast<const float4*>(&s_sc[tg][kofs + 4 * w4]);
+              r4[0] = rv.x; r4[1] = rv.y; r4[2] = rv.z; r4[3] = rv.w;
+              s4[0] = sv.x; s4[1] = sv.y; s4[2] = sv.z; s4[3] = sv.w;
+            } else {
+              const float rj = s_rc[tg][g + RG * jj], sj = s_sc[tg][g + RG * jj];
+#pragma unroll
+              for (int e = 0; e < 4; ++e) { r4[e] = rj; s4[e] = sj; }
+            }
+            const float2 y01 = __fmul2_rn(make_float2(S[jj][4 * w4], S[jj][4 * w4 + 1]), make_float2(r4[0], r4[1]));
+            const float2 y23 = __fmul2_rn(make_float2(S[jj][4 * w4 + 2], S[jj][4 * w4 + 3]), make_float2(r4[2], r4[3]));
+            codes[jj][w4] = float_to_i8x4(y01.x, y01.y, y23.x, y23.y);
+            if (keep) {
+              float c4[4];
+              i8x4_to_float(codes[jj][w4], c4);
+#pragma unroll
+              for (int e = 0; e < 4; ++e) S[jj][4 * w4 + e] = __fmul_rn(c4[e], s4[e]);
+            }
+          }
+        }
       }
       if constexpr (SDT != ST_F32) {
         if (stored_readout) {
@@ -442,7 +571,10 @@ step_seq(const StepParams p) {
           }
         }
       }
-      if (writer) st_out1(p.out, ((int64_t)tok * p.HV + hv) * V + out_col, o_mine, out_bf16);
+      if (writer) {
+        if constexpr (I8) s_ot[tt][out_col - v0] = o_mine;  // R o; rotated back after the chunk
+        else st_out1(p.out, ((int64_t)tok * p.HV + hv) * V + out_col, o_mine, out_bf16);
+      }
       if constexpr (IDX == IDX_PAGED) {
         // a page that fills inside a multi-token suffix keeps this state
         if (u.T > 1) {
@@ -456,6 +588,14 @@ step_seq(const StepParams p) {
       }
     }
     __syncthreads();  // the next chunk's prologue overwrites the token buffers
+    if constexpr (I8) {
+      // the chunk's outputs back from the rotated basis: one warp per (token, group)
+      for (int pr = warp; pr < nt * NG; pr += NW) {
+        const int tt = pr / NG, gi = pr % NG;
+        const float o = __fmul_rn(fwht_lanes(s_ot[tt][32 * gi + lane], lane), inv_sqrt32());
+        st_out1(p.out, ((int64_t)(t0 + tt) * p.HV + hv) * V + v0 + 32 * gi + lane, o, out_bf16);
+      }
+    }
   }
 
   // ---- store the state once, after the last token

@@ -26,8 +26,9 @@
  * flashinfer.gdn_paged.gated_delta_rule_decode_paged (description,
  * Parameters, Notes); max.nn.state_space.kda_decode (description,
  * Parameters, Raises); modelopt.torch.quantization.linear_attention.config
- * (LinearAttentionConfig state.block_v, LinearAttentionDecodeConfig readout)
- * and ...linear_attention.decode (recurrent_decode: fp8_e4m3, block_v=64;
+ * (LinearAttentionConfig state.block_v and the int8_hadamard32 decode codec,
+ * LinearAttentionDecodeConfig readout and state_codec) and
+ * ...linear_attention.decode (recurrent_decode: fp8_e4m3, block_v=64;
  * recurrent_decode_reference: an empty call performs no write).
  *
  * Conventions of every entry point:
@@ -78,7 +79,10 @@ typedef enum gdn_status {
 typedef enum gdn_dtype {
   GDN_F32 = 0,
   GDN_BF16 = 1,
-  GDN_FP8_E4M3 = 2 /* state only: codes + one fp32 scale per [K, block_v] tile */
+  GDN_FP8_E4M3 = 2, /* state only: codes + one fp32 scale per [K, block_v] tile */
+  GDN_INT8_H32 = 3  /* state only: int8_hadamard32, int8 codes of each
+                       (key channel, 32 values) group rotated by H32/sqrt(32),
+                       + one fp32 scale per group */
 } gdn_dtype;
 
 typedef enum gdn_index_dtype { GDN_I32 = 0, GDN_I64 = 1 } gdn_index_dtype;
@@ -87,7 +91,7 @@ typedef enum gdn_index_dtype { GDN_I32 = 0, GDN_I64 = 1 } gdn_index_dtype;
  * V_FIRST: [V][K], K contiguous (the paged pool's [num_pages, HV, V, K]). */
 typedef enum gdn_layout { GDN_K_FIRST = 0, GDN_V_FIRST = 1 } gdn_layout;
 
-/* Which state o is read from when the state is stored in bf16 or fp8:
+/* Which state o is read from when the state is stored in bf16, fp8 or int8:
  * WORKING = the fp32 state before it is rounded to its storage format,
  * STORED = the state after that rounding. Equal for fp32 states. */
 typedef enum gdn_readout { GDN_READOUT_WORKING = 0, GDN_READOUT_STORED = 1 } gdn_readout;
@@ -103,12 +107,21 @@ typedef enum kda_beta_mode { KDA_BETA_LOGITS = 0, KDA_BETA_PROBABILITY = 1 } kda
 
 /* The recurrent-state pool.
  *  data:      [num_slots, HV, K, V] logically, stored per `layout` in
- *             `dtype` (fp8: one uint8 E4M3 code per element).
- *  scales:    fp8 only: [num_slots, HV, V / block_v] fp32, one per
- *             [K, block_v] tile; NULL otherwise.
- *  block_v:   fp8 tile width along V (64); ignored for fp32/bf16.
+ *             `dtype` (fp8: one uint8 E4M3 code per element; int8: one int8
+ *             code per element).
+ *  scales:    fp8: [num_slots, HV, V / block_v] fp32, one per [K, block_v]
+ *             tile. int8_hadamard32: [num_slots, HV, V / 32, K] fp32, one
+ *             per (32-value group, key channel), for either layout, 16-byte
+ *             aligned. NULL otherwise.
+ *  block_v:   fp8 tile width along V (64); ignored for the other dtypes.
  * fp8 states are decoded as code * scale when read and re-encoded with a
- * fresh scale (amax / 448) after every token. */
+ * fresh scale (amax / 448) after every token.
+ * int8_hadamard32 (ModelOpt linear-attention config: the decode codec whose
+ * scales are fixed to one key channel and 32 values): for key channel k and
+ * values 32g..32g+31, y = R x with R = H32 / sqrt(32) (Sylvester order,
+ * symmetric, R R = I), s = amax|y| / 127, code = y / s rounded to nearest
+ * even; decoding is R (code * s). Re-encoded after every token. Needs
+ * V % 64 == 0 (else GDN_ERR_UNSUPPORTED). */
 typedef struct gdn_state_pool {
   void* data;
   float* scales;
@@ -128,10 +141,10 @@ typedef struct gdn_state_pool {
  *                written in place after the last token.
  *  out      [B, T, HV, V]  out_dtype (F32 or BF16)
  * Constraints: HV % H == 0; K and V in {32, 64, 128, 256}; fp8 state needs
- * block_v == 64 and V % 64 == 0.
+ * block_v == 64 and V % 64 == 0; int8_hadamard32 state needs V % 64 == 0.
  * T > 1 runs the tokens of each sequence in order with the state held on
- * chip (a short suffix); bf16/fp8 states pass through their storage format
- * after every token. */
+ * chip (a short suffix); bf16/fp8/int8 states pass through their storage
+ * format after every token. */
 typedef struct gdn_decode_slots_params {
   int32_t struct_size; /* sizeof(gdn_decode_slots_params) */
   int32_t B, T, H, HV, K, V;
@@ -260,7 +273,7 @@ int gdn_paged_decode_slots(const void* page_indices, const void* page_indptr,
  * q and k are always L2-normalised and q scaled by 1/sqrt(K). A sequence of
  * zero tokens leaves its slot untouched. gate_mode KDA_GATE_SAFE returns
  * GDN_ERR_UNSUPPORTED (its lower bound is not defined by the source).
- * State dtypes: F32 or BF16. */
+ * State dtypes: any gdn_dtype, with the pool rules above. */
 typedef struct kda_decode_varlen_params {
   int32_t struct_size; /* sizeof(kda_decode_varlen_params) */
   int32_t B, total_tokens, Hk, HV, K, V;
@@ -294,6 +307,25 @@ int gdn_state_quantize_fp8(const float* src, uint8_t* codes, float* scales, int6
 int gdn_state_dequantize_fp8(const uint8_t* codes, const float* scales, float* dst,
                              int64_t n_states, int32_t K, int32_t V, int32_t block_v,
                              int32_t layout, gdn_stream_t stream);
+
+/* int8_hadamard32 codec over n_states states of [K, V] (stored per layout),
+ * the pool's code format on its own (see gdn_state_pool). Everything in
+ * binary32 with one fixed rounding order, so results are reproducible bit
+ * for bit: the 32 values of a group are rotated by the fast Walsh-Hadamard
+ * butterflies of span 1, 2, 4, 8, 16 ((a, b) -> (a + b, a - b)), each then
+ * multiplied by the binary32 nearest 1/sqrt(32); s = amax / 127 and
+ * r = 1 / s round to nearest; code = y * r (rounded product) rounded to the
+ * nearest integer, ties to even (clamped to +-127, which finite inputs
+ * never reach). A group whose amax is 0, or whose r is not finite, stores
+ * s = 0 and codes 0. Decoding multiplies code * s (rounded) and applies the
+ * same butterflies and product.
+ *  src/dst [n_states, K, V] or [n_states, V, K] fp32; codes same shape
+ *  int8; scales [n_states, V / 32, K] fp32. All pointers 16-byte aligned. */
+int gdn_state_quantize_int8h32(const float* src, int8_t* codes, float* scales, int64_t n_states,
+                               int32_t K, int32_t V, int32_t layout, gdn_stream_t stream);
+int gdn_state_dequantize_int8h32(const int8_t* codes, const float* scales, float* dst,
+                                 int64_t n_states, int32_t K, int32_t V, int32_t layout,
+                                 gdn_stream_t stream);
 
 /* Static description of a status code (never NULL). */
 const char* gdn_status_string(int status);

@@ -6,7 +6,9 @@ Tolerances (max relative error per (sequence, value head) slice,
 max|x - ref| / max|ref|): fp32 state 1e-4 on outputs and states; bf16 state
 2e-2; fp8 state: outputs 1e-4 (working readout reads the fp32 state), stored
 codes within one E4M3 step of the oracle's after dequantisation and >= 99.9%
-identical. bf16 outputs add the bf16 rounding of the output, 2^-8.
+identical; int8_hadamard32 state: outputs 1e-4, scales within 1e-5, codes
+within one code step (compared as code * scale, the rotated values) and
+>= 99.9% identical. bf16 outputs add the bf16 rounding of the output, 2^-8.
 """
 
 from __future__ import annotations
@@ -21,7 +23,8 @@ import workloads as W
 from oracle import formats
 from oracle import gdn as O
 
-TOL = {"f32": 1e-4, "bf16": 2e-2, "fp8_e4m3": 1e-4}
+TOL = {"f32": 1e-4, "bf16": 2e-2, "fp8_e4m3": 1e-4, "int8_hadamard32": 1e-4}
+CODED = ("fp8_e4m3", "int8_hadamard32")
 BF16_OUT = 2.0 ** -8
 # fp8 state read out from the STORED (re-encoded) state: where the two fp32
 # working states straddle an E4M3 rounding boundary the two sides store
@@ -34,12 +37,14 @@ TOL_FP8_STORED = 1e-2
 # token, so a code that lands on the neighbouring E4M3 value on one side
 # (an fp32 rounding difference at a rounding boundary) is carried into the
 # later tokens' outputs; the same one-step bound applies. The stored codes
-# are still held to one step and >= 99.9% identical.
+# are still held to one step and >= 99.9% identical. The int8_hadamard32
+# state has the same mechanism with a step of amax / 127 per group, far
+# below an E4M3 step at the group's top, so the same bound holds.
 TOL_FP8_RUN = 1e-2
 
 
 def out_tol(state_dtype, readout, multi_token):
-    if state_dtype == "fp8_e4m3" and (readout == "stored" or multi_token):
+    if state_dtype in CODED and (readout == "stored" or multi_token):
         return TOL_FP8_RUN
     return TOL[state_dtype]
 
@@ -99,6 +104,23 @@ def check_state(pool_after: np.ndarray, scales_after, writes, state_dtype: str, 
             e = slice_rel_err(got, st_ref)
         elif state_dtype == "bf16":
             e = slice_rel_err(formats.bf16_bits_to_f32(got), formats.bf16_bits_to_f32(st_ref))
+        elif state_dtype == "int8_hadamard32":
+            sc_got = scales_after[slot, hv]
+            assert np.allclose(sc_got, sc_ref, rtol=1e-5, atol=0), (slot, hv)
+            kv_got = O._to_kv(got, layout)
+            kv_ref = O._to_kv(st_ref, layout)
+            s_got = np.repeat(sc_got.T.astype(np.float64), 32, axis=1)      # [K, V]
+            s_ref = np.repeat(sc_ref.T.astype(np.float64), 32, axis=1)
+            rot_got = kv_got.astype(np.float64) * s_got
+            rot_ref = kv_ref.astype(np.float64) * s_ref
+            lim = 1.002 * np.maximum(s_got, s_ref) + 1e-30                  # one code step
+            assert np.all(np.abs(rot_got - rot_ref) <= lim), f"int8 state (slot={slot}, hv={hv}) off by > 1 step"
+            n_codes += got.size
+            n_same += int(np.sum(got == st_ref))
+            e = slice_rel_err(formats.dequantize_state_h32(kv_got, sc_got),
+                              formats.dequantize_state_h32(kv_ref, sc_ref))
+            worst = max(worst, e)
+            continue
         else:
             sc_got = scales_after[slot, hv]
             assert np.allclose(sc_got, sc_ref, rtol=1e-5, atol=0), (slot, hv, sc_got, sc_ref)
@@ -119,7 +141,7 @@ def check_state(pool_after: np.ndarray, scales_after, writes, state_dtype: str, 
         worst = max(worst, e)
         assert e <= TOL[state_dtype], f"state (slot={slot}, hv={hv}): rel err {e:.3g}"
     if n_codes:
-        assert n_same / n_codes >= 0.999, f"only {n_same / n_codes:.5f} of fp8 codes identical"
+        assert n_same / n_codes >= 0.999, f"only {n_same / n_codes:.5f} of {state_dtype} codes identical"
     return worst
 
 
@@ -137,7 +159,7 @@ def check_untouched(pool_before: np.ndarray, pool_after: np.ndarray, written_key
 
 
 def check_stored_readout(out_gpu, t, idx, pool_after, scales_after, units, layout, scale, use_qk_l2norm,
-                         num_slots, block_v=64):
+                         num_slots, block_v=64, state_dtype="fp8_e4m3"):
     """Validity of a stored readout: the last token's output is q^ times the
     state the kernel stored (decoded by the oracle's codec)."""
     K = t["q"].shape[-1]
@@ -148,7 +170,7 @@ def check_stored_readout(out_gpu, t, idx, pool_after, scales_after, units, layou
         if not 0 <= s < num_slots:
             continue
         qh, _ = O.prepare_qk(t["q"][b, -1, O.key_head_of(hv, H, HV)], t["k"][b, -1, 0], sc, use_qk_l2norm)
-        S = O.load_state(pool_after[s, hv], layout, "fp8_e4m3", scales_after[s, hv], block_v)
+        S = O.load_state(pool_after[s, hv], layout, state_dtype, scales_after[s, hv], block_v)
         e = slice_rel_err(out_gpu[b, -1, hv], qh @ S)
         assert e <= 1e-4, f"stored readout (b={b}, hv={hv}) is not q^T of the stored state: {e:.3g}"
 
@@ -192,9 +214,9 @@ def gdn_slots_case(seed, B, T, H, HV, K, V, num_slots, layout="V_FIRST", state_d
     todo = [(b, hv) for b in range(B) for hv in range(HV)] if units is None else units
     res["out_err"] = check_outputs(res["out"], ref_out, todo, lambda x, b, hv: x[b, :, hv, :],
                                    out_tol(state_dtype, readout, T > 1), out_dtype)
-    if state_dtype == "fp8_e4m3" and readout == "stored":
+    if state_dtype in CODED and readout == "stored":
         check_stored_readout(res["out"], t, idx, after, sc_after, todo, layout, scale, use_qk_l2norm,
-                             num_slots, block_v)
+                             num_slots, block_v, state_dtype)
     res["state_err"] = check_state(after, sc_after, writes, state_dtype, layout, block_v)
     written = {(s, hv) for s in live for hv in range(HV)} if T > 0 else set()
     check_untouched(before, after, written, sc_before, sc_after)

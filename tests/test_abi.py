@@ -32,7 +32,8 @@ def declared_functions():
 def test_every_declared_symbol_is_exported(lib):
     names = declared_functions()
     assert {"gdn_decode_slots", "gdn_decode_paged", "gdn_paged_decode_slots", "kda_decode_varlen", "gdn_prefill_paged",
-            "gdn_state_quantize_fp8", "gdn_state_dequantize_fp8", "gdn_status_string"} <= set(names)
+            "gdn_state_quantize_fp8", "gdn_state_dequantize_fp8", "gdn_state_quantize_int8h32",
+            "gdn_state_dequantize_int8h32", "gdn_status_string"} <= set(names)
     for n in names:
         assert hasattr(lib, n), f"{n} is declared in include/gdn.h but not exported"
 
@@ -103,6 +104,10 @@ def _slots_params(**kw):
     (dict(pool_dtype=G.GDN_FP8_E4M3), G.GDN_ERR_INVALID_ARG),            # fp8 without scales
     (dict(pool_dtype=G.GDN_FP8_E4M3, pool_scales=FAKE, pool_block_v=32), G.GDN_ERR_UNSUPPORTED),
     (dict(pool_dtype=G.GDN_FP8_E4M3, pool_scales=FAKE, pool_block_v=48), G.GDN_ERR_INVALID_ARG),
+    (dict(pool_dtype=G.GDN_INT8_H32), G.GDN_ERR_INVALID_ARG),            # int8 without scales
+    (dict(pool_dtype=G.GDN_INT8_H32, pool_scales=FAKE + 4), G.GDN_ERR_INVALID_ARG),   # scales not 16-byte aligned
+    (dict(pool_dtype=G.GDN_INT8_H32, pool_scales=FAKE, V=32), G.GDN_ERR_UNSUPPORTED),
+    (dict(pool_dtype=4, pool_scales=FAKE), G.GDN_ERR_INVALID_ARG),
     (dict(q=FAKE + 4), G.GDN_ERR_INVALID_ARG),                           # misaligned
     (dict(out=None), G.GDN_ERR_INVALID_ARG),
     (dict(B=0), G.GDN_OK),                                               # nothing to do, no launch
@@ -159,6 +164,14 @@ def test_codec_validation(lib):
     assert f(FAKE, FAKE, FAKE, 1, 128, 100, 64, 1, None) == G.GDN_ERR_INVALID_ARG
     assert f(FAKE, FAKE, FAKE, 0, 128, 128, 64, 1, None) == G.GDN_OK
     assert lib.gdn_state_dequantize_fp8(FAKE, FAKE, FAKE, 1, 128, 128, 64, 7, None) == G.GDN_ERR_INVALID_ARG
+    q8, d8 = lib.gdn_state_quantize_int8h32, lib.gdn_state_dequantize_int8h32
+    assert q8(FAKE, FAKE, FAKE, 1, 128, 96, 1, None) == G.GDN_ERR_INVALID_ARG        # V not a head dim
+    assert q8(FAKE, FAKE, FAKE, 1, 128, 128, 2, None) == G.GDN_ERR_INVALID_ARG       # layout
+    assert q8(FAKE, FAKE + 8, FAKE, 1, 128, 128, 1, None) == G.GDN_ERR_INVALID_ARG   # codes misaligned
+    assert q8(FAKE, None, FAKE, 1, 128, 128, 0, None) == G.GDN_ERR_INVALID_ARG
+    assert q8(FAKE, FAKE, FAKE, 0, 128, 128, 0, None) == G.GDN_OK
+    assert d8(FAKE, FAKE, FAKE, -1, 128, 128, 0, None) == G.GDN_ERR_INVALID_ARG
+    assert d8(FAKE, FAKE, FAKE, 0, 32, 32, 1, None) == G.GDN_OK
     assert lib.gdn_paged_decode_slots(FAKE, FAKE, FAKE, 3, 4, 2, 8, 0, FAKE, None, None) == G.GDN_ERR_INVALID_ARG
     assert lib.gdn_paged_decode_slots(FAKE, FAKE, FAKE, 0, 4, 0, 8, 0, FAKE, None, None) == G.GDN_OK
 

@@ -1,0 +1,113 @@
+"""int8_hadamard32 state (one scale per key channel and 32 values, the
+ModelOpt linear-attention decode codec): the codec calls bit for bit against
+the oracle, and every decode path on an int8 pool against the oracle."""
+
+import numpy as np
+import pytest
+import torch
+
+import gated_delta_rule_80_b200 as G
+import workloads as W
+from gdn_cases import dev, gdn_paged_case, gdn_prefill_case, gdn_slots_case, kda_case
+from oracle import gdn as O
+
+pytestmark = [pytest.mark.gpu,
+              pytest.mark.skipif(not torch.cuda.is_available(), reason="needs a CUDA device")]
+
+I8 = "int8_hadamard32"
+
+
+def _codec_states(N, K, V, layout, seed=91):
+    """States with the codec's edge cases in the first few: a zero state, a
+    state of one spike per group, an all-negative state, values near the
+    bottom of binary32 (r overflows), groups whose rotated values take two
+    magnitudes only, and a spread of magnitudes across key channels."""
+    r = np.random.default_rng(seed)
+    kv = (r.standard_normal((N, K, V)) * 0.1).astype(np.float32)
+    kv[0] = 0.0
+    kv[1] = 0.0
+    kv[1, :, ::32] = r.standard_normal((K, V // 32)).astype(np.float32)
+    kv[2] = -np.abs(kv[2])
+    kv[3] = np.float32(1e-39)
+    kv[4, :, :] = 0.0
+    kv[4, :, 0::32] = 127.0 / np.sqrt(np.float32(32.0))
+    kv[4, :, 1::32] = np.float32(0.5) / np.sqrt(np.float32(32.0))
+    kv[5] *= np.exp(r.uniform(-20, 20, (K, 1))).astype(np.float32)
+    x = kv if layout == "K_FIRST" else np.ascontiguousarray(kv.transpose(0, 2, 1))
+    return x
+
+
+@pytest.mark.parametrize("layout", ["V_FIRST", "K_FIRST"])
+@pytest.mark.parametrize("K,V", [(128, 128), (32, 32), (64, 128), (256, 256), (256, 64), (32, 256)])
+def test_int8h32_codec_bit_exact(layout, K, V):
+    x = _codec_states(8, K, V, layout)
+    codes, scales = G.gdn_state_quantize_int8h32(dev(x), layout=layout)
+    ref_codes, ref_scales = O.state_quantize_h32(x, layout)
+    assert np.array_equal(scales.cpu().numpy().view(np.uint32), ref_scales.view(np.uint32))
+    assert np.array_equal(codes.cpu().numpy(), ref_codes)
+    assert not codes[0].any() and not scales[0].any() and not scales[3].any()
+    deq = G.gdn_state_dequantize_int8h32(codes, scales, layout=layout).cpu().numpy()
+    ref_deq = O.state_dequantize_h32(ref_codes, ref_scales, layout)
+    assert np.array_equal(deq.view(np.uint32), ref_deq.view(np.uint32))
+
+
+@pytest.mark.parametrize("layout", ["V_FIRST", "K_FIRST"])
+@pytest.mark.parametrize("T", [1, 3])
+def test_int8h32_slots(layout, T):
+    gdn_slots_case(92 + T, B=5, T=T, H=2, HV=4, K=128, V=128, num_slots=7, layout=layout, state_dtype=I8)
+
+
+@pytest.mark.parametrize("K,V", [(32, 64), (64, 128), (128, 64), (256, 256), (256, 64), (32, 256)])
+@pytest.mark.parametrize("layout", ["V_FIRST", "K_FIRST"])
+def test_int8h32_head_dims(K, V, layout):
+    gdn_slots_case(94, B=3, T=2, H=1, HV=2, K=K, V=V, num_slots=4, layout=layout, state_dtype=I8, in_dtype="f32")
+
+
+@pytest.mark.parametrize("layout", ["V_FIRST", "K_FIRST"])
+@pytest.mark.parametrize("T", [1, 2])
+def test_int8h32_stored_readout(layout, T):
+    gdn_slots_case(95, B=4, T=T, H=1, HV=2, K=64, V=128, num_slots=6, layout=layout, state_dtype=I8,
+                   readout="stored")
+
+
+def test_int8h32_bf16_outputs_padded_int64():
+    r = gdn_slots_case(96, B=4, T=1, H=1, HV=2, K=128, V=128, num_slots=5, state_dtype=I8, out_dtype="bf16",
+                       index_dtype="i64", indices=[3, -1, 0, 7])
+    assert r["err"] == 1            # slot 7 is out of range
+    assert not r["out"][1].any() and not r["out"][3].any()
+
+
+@pytest.mark.parametrize("layout", ["V_FIRST", "K_FIRST"])
+def test_int8h32_paged(layout):
+    gdn_paged_case(97, B=6, H=1, HV=2, K=128, V=128, page_size=8, max_len=60, n_share=2, share_pages=2,
+                   force_lens={0: 17, 1: 9}, state_dtype=I8, layout=layout)
+
+
+@pytest.mark.parametrize("layout", ["V_FIRST", "K_FIRST"])
+def test_int8h32_paged_suffix(layout):
+    gdn_paged_case(98, B=4, H=1, HV=2, K=64, V=128, page_size=4, max_len=40, n_share=0, share_pages=0,
+                   state_dtype=I8, T=6, layout=layout, min_len=6 + 2 * 4 + 1)
+
+
+@pytest.mark.parametrize("layout", ["V_FIRST", "K_FIRST"])
+def test_int8h32_prefill(layout):
+    r = gdn_prefill_case(99, B=5, H=1, HV=2, K=128, V=128, page_size=8, max_len=40, state_dtype=I8, layout=layout)
+    assert r["err"] == 0
+
+
+@pytest.mark.parametrize("layout", ["K_FIRST", "V_FIRST"])
+def test_int8h32_kda(layout):
+    kda_case(100, B=4, Hk=2, HV=2, K=128, V=128, num_slots=6, max_len=5, layout=layout, state_dtype=I8)
+
+
+def test_int8h32_large_batch_reduced():
+    w = W.WORKLOADS["int8"]
+    gdn_slots_case(w.seed, B=24, T=1, H=w.H, HV=w.HV, K=w.K, V=w.V, num_slots=64, state_dtype=I8)
+
+
+def test_int8h32_full_size_sampled():
+    w = W.WORKLOADS["int8"]
+    r = np.random.default_rng(101)
+    units = sorted({(int(b), int(h)) for b, h in zip(r.integers(0, w.B, 300), r.integers(0, w.HV, 300))})
+    gdn_slots_case(w.seed, w.B, w.T, w.H, w.HV, w.K, w.V, w.num_slots, state_dtype=I8,
+                   in_dtype="bf16", out_dtype="bf16", units=units)
