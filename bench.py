@@ -8,7 +8,7 @@ back in place. Steps rotate over 4 disjoint sets of 64 slots (512 MiB of
 state per cycle, 4x the L2), so no step finds its state in L2.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl b200|reference]
-                    [--workload slots|paged|kda|fp8|tiny]
+                    [--workload slots|paged|kda|fp8|int8|tiny|prefill]
 
 Prints one JSON line (rank 0). Under torchrun each rank runs its own batch
 on its own GPU (weak scaling; the sequences are independent, no data-path
@@ -50,7 +50,8 @@ def parse():
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["b200", "reference"], default="b200")
-    ap.add_argument("--workload", choices=["slots", "paged", "kda", "fp8", "tiny", "prefill"], default="slots")
+    ap.add_argument("--workload", choices=["slots", "paged", "kda", "fp8", "int8", "tiny", "prefill"],
+                    default="slots")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
@@ -172,7 +173,7 @@ def describe_slots(w: W.Workload) -> str:
 
 
 class SlotsRun:
-    """GDN slot pool, T=1 (the 'slots' and 'fp8' workloads)."""
+    """GDN slot pool, T=1 (the 'slots', 'fp8', 'int8' and 'tiny' workloads)."""
 
     def __init__(self, w: W.Workload, rank: int):
         import gated_delta_rule_80_b200 as G
@@ -190,8 +191,10 @@ class SlotsRun:
         self.idx = [torch.from_numpy(W.slot_indices(seed, w.B, w.num_slots, r).astype(np.int32)).cuda()
                     for r in range(self.n_rot)]
         self.out = torch.empty((w.B, w.T, w.HV, w.V), dtype=torch.bfloat16, device="cuda")
-        sb = {"f32": 4, "bf16": 2, "fp8_e4m3": 1}[w.state_dtype]
-        state = 2 * w.HV * w.K * w.V * sb + (2 * w.HV * (w.V // w.block_v) * 4 if w.state_dtype == "fp8_e4m3" else 0)
+        sb = {"f32": 4, "bf16": 2, "fp8_e4m3": 1, "int8_hadamard32": 1}[w.state_dtype]
+        # codes plus scales, each read and written once
+        sc_per_head = {"fp8_e4m3": (w.V // w.block_v) * 4, "int8_hadamard32": (w.V // 32) * w.K * 4}
+        state = 2 * w.HV * (w.K * w.V * sb + sc_per_head.get(w.state_dtype, 0))
         ib = 2 if w.in_dtype == "bf16" else 4
         io = (2 * w.H * w.K + w.HV * w.V + 2 * w.HV) * ib + w.HV * w.V * 2 + 4
         self.tokens_per_step = w.B * w.T
@@ -399,7 +402,7 @@ class PrefillRun:
 
 def make_run(name, rank):
     w = W.WORKLOADS.get(name)
-    if name in ("slots", "fp8", "tiny"):
+    if name in ("slots", "fp8", "int8", "tiny"):
         return SlotsRun(w, rank)
     if name == "paged":
         return PagedRun(w, rank)

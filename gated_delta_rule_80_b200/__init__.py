@@ -36,7 +36,7 @@ GDN_K_FIRST, GDN_V_FIRST = 0, 1
 GDN_READOUT_WORKING, GDN_READOUT_STORED = 0, 1
 KDA_GATE_ORIGINAL, KDA_GATE_SAFE = 0, 1
 KDA_BETA_LOGITS, KDA_BETA_PROBABILITY = 0, 1
-GDN_FLAG_SLOT_RANGE, GDN_FLAG_PAGE_RANGE, GDN_FLAG_PAGE_TABLE, GDN_FLAG_SEQLENS = 1, 2, 4, 8
+GDN_FLAG_SLOT_RANGE, GDN_FLAG_PAGE_RANGE, GDN_FLAG_PAGE_TABLE, GDN_FLAG_SEQLENS, GDN_FLAG_TIMEOUT = 1, 2, 4, 8, 16
 
 _LAYOUTS = {"K_FIRST": GDN_K_FIRST, "V_FIRST": GDN_V_FIRST}
 _READOUTS = {"working": GDN_READOUT_WORKING, "stored": GDN_READOUT_STORED}

@@ -15,6 +15,7 @@
 
 #include "../../include/gdn.h"
 #include "gdn_seq.cuh"
+#include "gdn_pipe_i8.cuh"
 
 using namespace gdn;
 
@@ -90,6 +91,36 @@ int launch_tile1(StepParams p, int B, cudaStream_t s) {
   return launch_status();
 }
 
+// Single-token GDN decode on a V_FIRST int8_hadamard32 pool: persistent
+// CTAs (as many as fit on the device at once) over the (sequence, value head,
+// scale group) tiles.
+template <int K, int IDX>
+int launch_pipe_i8(StepParams p, int B, cudaStream_t s) {
+  using PS = PipeI8Shape<K>;
+  static int resident[64] = {0};  // CTAs per SM, per device
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64 ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+    cudaGetLastError();
+    return GDN_ERR_CUDA;
+  }
+  if (resident[dev] == 0) {
+    int n = 0;
+    if (cudaFuncSetAttribute(step_pipe_i8<K, IDX>, cudaFuncAttributeMaxDynamicSharedMemorySize, PS::SMEM) !=
+            cudaSuccess ||
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, step_pipe_i8<K, IDX>, PS::NT, PS::SMEM) != cudaSuccess ||
+        n < 1) {
+      cudaGetLastError();
+      return GDN_ERR_CUDA;
+    }
+    resident[dev] = n;
+  }
+  const int64_t n_tiles = (int64_t)B * p.HV * (p.V / PS::VT);
+  const int64_t grid = std::min<int64_t>(n_tiles, (int64_t)sms * resident[dev]);
+  step_pipe_i8<K, IDX><<<static_cast<unsigned>(grid), PS::NT, PS::SMEM, s>>>(p, n_tiles);
+  return launch_status();
+}
+
 // T >= 1 tokens per unit, either layout: the chunked-prologue kernel.
 template <int L, int SDT, int K, int GATE, int IDX, int NW>
 int launch_seq_nw(StepParams p, int B, cudaStream_t s) {
@@ -105,8 +136,11 @@ int launch_one(StepParams p, int B, cudaStream_t s) {
   p.G = p.HV / p.H;
   if (B > 65535) return GDN_ERR_INVALID_ARG;  // grid z
   constexpr bool CODED = (SDT == ST_FP8 || SDT == ST_I8H);
-  if constexpr (L == L_VFIRST && GATE == GATE_SCALAR && SDT != ST_I8H) {
-    if (p.T == 1) return launch_tile1<SDT, K, IDX>(p, B, s);
+  if constexpr (L == L_VFIRST && GATE == GATE_SCALAR) {
+    if (p.T == 1) {
+      if constexpr (SDT == ST_I8H) return launch_pipe_i8<K, IDX>(p, B, s);
+      else return launch_tile1<SDT, K, IDX>(p, B, s);
+    }
   }
   if constexpr (L == L_KFIRST) {
     constexpr int VTW = (K == 256) ? 8 : 16;  // columns per warp
