@@ -415,25 +415,29 @@ def make_run(name, rank):
 # roofline bookkeeping
 # ----------------------------------------------------------------------------
 
-def source_digest():
+def source_digest(files=None):
+    """First 16 hex of the sha256 over the named kernel sources (all of csrc
+    when none are named), in sorted order."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "gated_delta_rule_80_b200", "csrc")
-    for f in sorted(os.listdir(csrc)):
-        if f.endswith((".cu", ".cuh")):
-            h.update(open(os.path.join(csrc, f), "rb").read())
+    names = sorted(files) if files else sorted(f for f in os.listdir(csrc) if f.endswith((".cu", ".cuh")))
+    for f in names:
+        h.update(open(os.path.join(csrc, f), "rb").read())
     return h.hexdigest()[:16]
 
 
 def profiled_traffic(workload):
     """DRAM bytes per launch from the committed ncu summary of this workload,
-    or None when the kernel sources changed since it was taken."""
+    or None when the kernel sources it names changed since it was taken."""
     path = os.path.join(PROFILES, f"gdn_decode_{workload}_ncu.md")
     if not os.path.exists(path):
         return None
     text = open(path).read()
     dig = re.search(r"source_digest:\s*([0-9a-f]+)", text)
     tb = re.search(r"dram_bytes_per_launch:\s*([0-9.e+]+)", text)
-    if not dig or not tb or dig.group(1) != source_digest():
+    fl = re.search(r"source_files:\s*([^\n]+)", text)
+    files = fl.group(1).split() if fl else None
+    if not dig or not tb or dig.group(1) != source_digest(files):
         return None
     return float(tb.group(1))
 
