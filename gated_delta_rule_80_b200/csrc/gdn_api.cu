@@ -16,6 +16,7 @@
 #include "../../include/gdn.h"
 #include "gdn_seq.cuh"
 #include "gdn_pipe_i8.cuh"
+#include "gdn_chunk_tc.cuh"
 
 using namespace gdn;
 
@@ -118,6 +119,29 @@ int launch_pipe_i8(StepParams p, int B, cudaStream_t s) {
   const int64_t n_tiles = (int64_t)B * p.HV * (p.V / PS::VT);
   const int64_t grid = std::min<int64_t>(n_tiles, (int64_t)sms * resident[dev]);
   step_pipe_i8<K, IDX><<<static_cast<unsigned>(grid), PS::NT, PS::SMEM, s>>>(p, n_tiles);
+  return launch_status();
+}
+
+// Paged prefill on the tensor cores (fp32 V_FIRST pages, K = V = 128, bf16
+// token inputs, page_size a multiple of 64): one CTA per (value head, sequence).
+int launch_prefill_tc(StepParams p, int B, cudaStream_t s) {
+  static bool ready[64] = {false};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+    cudaGetLastError();
+    return GDN_ERR_CUDA;
+  }
+  if (!ready[dev]) {
+    if (cudaFuncSetAttribute(prefill_chunk_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, ChunkTC::SMEM) !=
+        cudaSuccess) {
+      cudaGetLastError();
+      return GDN_ERR_CUDA;
+    }
+    ready[dev] = true;
+  }
+  if (B > 65535) return GDN_ERR_INVALID_ARG;  // grid y
+  p.G = p.HV / p.H;
+  prefill_chunk_tc<<<dim3(p.HV, B), ChunkTC::NT, ChunkTC::SMEM, s>>>(p);
   return launch_status();
 }
 
@@ -517,6 +541,9 @@ int gdn_prefill_paged(const gdn_prefill_paged_params* p, gdn_stream_t stream) {
   k.flags = (p->in_dtype == GDN_BF16 ? F_IN_BF16 : 0) | (p->out_dtype == GDN_BF16 ? F_OUT_BF16 : 0) |
             (p->index_dtype == GDN_I64 ? F_IDX64 : 0) | (p->use_qk_l2norm ? F_L2NORM : 0) | F_VARLEN |
             (p->readout == GDN_READOUT_STORED ? F_READOUT_STORED : 0);
+  if (p->pool.dtype == GDN_F32 && p->pool.layout == GDN_V_FIRST && p->K == ChunkTC::D && p->V == ChunkTC::D &&
+      p->in_dtype == GDN_BF16 && p->page_size % ChunkTC::C == 0)
+    return launch_prefill_tc(k, p->B, reinterpret_cast<cudaStream_t>(stream));
   return launch_step<GATE_SCALAR, IDX_PAGED>(k, p->pool, p->K, p->B, reinterpret_cast<cudaStream_t>(stream));
 }
 

@@ -1,0 +1,525 @@
+// Paged prefill of fp32 states on the tensor cores: the chunked form of the
+// gated delta rule, 64 tokens per chunk, one CTA per (sequence, value head).
+//
+// Within a chunk (tokens t = 0..63 of the page-aligned chunk, g_t the
+// inclusive prefix sum of log alpha, S0 the state before the chunk):
+//     A_ts = beta_t (k^_t . k^_s) e^{g_t - g_s}      (s < t)
+//     P_ts = (q^_t . k^_s) e^{g_t - g_s}             (s <= t)
+//     R_t  = beta_t (v_t - e^{g_t} k^_t S0)
+//     (I + A) U = R                                  (forward substitution)
+//     o_t  = e^{g_t} q^_t S0 + sum_{s<=t} P_ts U_s
+//     S_C  = e^{g_C} S0 + sum_t e^{g_C - g_t} k^_t U_t^T
+// which is the scan of single steps (u_t = U_t) written for a block of
+// tokens (Circuit.LLM.Mixer "Gated memory": a prefill is the steps in order).
+//
+// The state is kept transposed (rows = value index, the V_FIRST page row) in
+// tensor memory as an fp32 accumulator. Three products run on tcgen05:
+//     G1   = S0^T [K ; Q]^T     (128 x 128 x 128: k S0 and q S0 of all tokens)
+//     Gram = [K ; Q] K^T        (128 x 64 x 128)
+//     S_C^T += (diag(w) U)^T K  (128 x 128 x 64, w_t = |k_t|^-1 e^{g_C - g_t})
+// with raw bf16 k and q rows as operands (their norms are applied to the
+// results) and the fp32 operands S0^T and (diag(w) U)^T split into three
+// bf16 terms each (hi + mid + lo carries 24 bits), so every product is exact
+// and the accumulation is fp32. The small triangular work (A, P, the
+// forward substitution, the outputs) runs on the CUDA cores: each of the two
+// warpgroups has one thread per value column v and takes half of the
+// columns, tokens or rows of every phase.
+//
+// Chunks are aligned to absolute token positions (multiples of 64), so with
+// page_size a multiple of 64 every page end is a chunk end; slots of a chunk
+// outside the run are padding (k = q = v = 0, alpha = 1, beta = 0), which
+// leaves the state and the other tokens unchanged.
+#pragma once
+
+#include "gdn_device.cuh"
+#include "gdn_umma.cuh"
+
+namespace gdn {
+
+struct ChunkTC {
+  static constexpr int C = 64;    // tokens per chunk
+  static constexpr int D = 128;   // K = V
+  static constexpr int NT = 256;  // two warpgroups; thread v of each owns value column v / tensor-memory lane v
+  // dynamic shared memory (bytes)
+  static constexpr uint32_t KQ = 0;               // 2 x [128 rows (k then q tokens) x 128] bf16, K-major
+  static constexpr uint32_t KQ_BYTES = 2 * C * D * 2;
+  static constexpr uint32_t VB = 2 * KQ_BYTES;    // 2 x [64 tokens x 128] bf16 row-major
+  static constexpr uint32_t V_BYTES = C * D * 2;
+  static constexpr uint32_t S3 = VB + 2 * V_BYTES;  // 3 x [128 x 128] bf16, K-major: S0^T split
+  static constexpr uint32_t S3_BYTES = D * D * 2;
+  // after G1 the S3 region holds the chunk's update operands and A, P
+  static constexpr uint32_t UT3 = S3;                 // 3 x [128 x 64] bf16, K-major: (diag(w) U)^T split
+  static constexpr uint32_t UT_BYTES = D * C * 2;
+  static constexpr uint32_t KT = UT3 + 3 * UT_BYTES;  // [128 x 64] bf16, K-major: K^T
+  static constexpr int AS = C + 4;                    // row stride of A and P (floats), staggers banks
+  static constexpr uint32_t AM = KT + UT_BYTES;       // [64 x AS] fp32
+  static constexpr uint32_t PM = AM + C * AS * 4;     // [64 x AS] fp32
+  static constexpr uint32_t SMEM = (PM + C * AS * 4 > S3 + 3 * S3_BYTES) ? PM + C * AS * 4 : S3 + 3 * S3_BYTES;
+  // tensor memory columns
+  static constexpr uint32_t T_ST = 0, T_G1 = 128, T_GR = 256, T_COLS = 512;
+};
+
+// Round to bf16 (nearest, ties to even) with integer operations: the result
+// is the float whose low 16 bits are zero. Finite inputs only.
+__device__ __forceinline__ float bf16_rne(float x) {
+  const uint32_t u = __float_as_uint(x);
+  return __uint_as_float((u + 0x7FFFu + ((u >> 16) & 1u)) & 0xFFFF0000u);
+}
+
+// x = hi + mid + lo, each a bf16 (as floats); x - hi and the next residual
+// are exact in binary32
+__device__ __forceinline__ void split_bf16x3(float x, float& h, float& m, float& l) {
+  h = bf16_rne(x);
+  const float r = x - h;
+  m = bf16_rne(r);
+  l = bf16_rne(r - m);
+}
+
+// 8 bf16-valued floats -> 16 bytes of bf16
+__device__ __forceinline__ uint4 pack_bf16x8(const float* x) {
+  uint32_t w[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) w[i] = __byte_perm(__float_as_uint(x[2 * i]), __float_as_uint(x[2 * i + 1]), 0x7632);
+  return make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+__device__ __forceinline__ void cp_async16(void* dst, const void* src, bool valid) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_addr(dst)), "l"(src),
+               "r"(valid ? 16 : 0)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+
+// The token inputs of the chunk starting at absolute position `base` into
+// input buffer `buf`: k rows and q rows into the [K ; Q] operand tile, v rows
+// row-major; slots outside [pos_lo, pos_hi) are zero filled.
+__device__ __forceinline__ void chunk_issue_loads(const StepParams& p, unsigned char* sm, int buf, int64_t base,
+                                                  int64_t pos_lo, int64_t pos_hi, int64_t tok_lo, int h, int hv) {
+  using CT = ChunkTC;
+  unsigned char* kq = sm + CT::KQ + buf * CT::KQ_BYTES;
+  unsigned char* vv = sm + CT::VB + buf * CT::V_BYTES;
+  for (int id = threadIdx.x; id < 3 * CT::C * 16; id += CT::NT) {
+    const int which = id / (CT::C * 16), rem = id % (CT::C * 16), j = rem / 16, piece = rem % 16;
+    const int64_t pos = base + j;
+    const bool valid = pos >= pos_lo && pos < pos_hi;
+    const int64_t tok = tok_lo + (pos - pos_lo);
+    const char* src = reinterpret_cast<const char*>(p.q);  // any valid address; no bytes are read when zero filling
+    unsigned char* dst;
+    if (which < 2) {
+      dst = kq + kmajor_offset(which * CT::C + j, 8 * piece, CT::D);
+      if (valid) src = reinterpret_cast<const char*>(which == 0 ? p.k : p.q) + ((tok * p.H + h) * CT::D) * 2 + piece * 16;
+    } else {
+      dst = vv + j * (CT::D * 2) + piece * 16;
+      if (valid) src = reinterpret_cast<const char*>(p.v) + ((tok * p.HV + hv) * CT::D) * 2 + piece * 16;
+    }
+    cp_async16(dst, src, valid);
+  }
+  cp_async_commit();
+}
+
+__global__ void __launch_bounds__(ChunkTC::NT, 1) prefill_chunk_tc(const StepParams p) {
+  using CT = ChunkTC;
+  constexpr int C = CT::C, D = CT::D;
+  extern __shared__ __align__(1024) unsigned char sm[];
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ uint32_t s_tmem;
+  __shared__ double s_g[C];
+  __shared__ double s_wsum;
+  __shared__ float s_beta[C], s_ik[C], s_iq[C];
+  __shared__ float s_egk[C], s_egq[C], s_wc[C];  // e^{g_t} |k_t|^-1, e^{g_t} scale |q_t|^-1, |k_t|^-1 e^{g_C - g_t}
+  __shared__ float s_nrm[D];                     // the second warpgroup's half of each row's sum of squares
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int wg = tid >> 7;      // warpgroup: splits the columns, tokens or rows of each phase
+  const int v = tid & (D - 1);  // value column, tensor-memory lane and tile row of this thread
+  const int hv = blockIdx.x, b = blockIdx.y;
+  const int h = hv / p.G;
+  const bool in_bf16 = (p.flags & F_IN_BF16) != 0;
+  const bool out_bf16 = (p.flags & F_OUT_BF16) != 0;
+
+  const Unit u = resolve_unit<IDX_PAGED>(p, b);
+  if (tid == 0) raise_err(p.err, u.err);
+  if (u.status == U_SKIP || u.tok1 <= u.tok0) return;
+  if (u.status == U_PAD) {
+    if (wg == 0)
+      for (int tok = u.tok0; tok < u.tok1; ++tok) st_out1(p.out, ((int64_t)tok * p.HV + hv) * D + v, 0.0f, out_bf16);
+    return;
+  }
+  const int64_t n = u.tok1 - u.tok0;
+  const int64_t pos_lo = u.L - n, pos_hi = u.L;
+  const int64_t base0 = (pos_lo / C) * C;
+  const int nchunks = static_cast<int>((pos_hi - base0 + C - 1) / C);
+  const int64_t head = (int64_t)D * D;  // floats of one (page, head) state
+  float* pool = reinterpret_cast<float*>(p.pool);
+
+  if (tid == 0) {
+    mbar_init(&bar, 1);
+    mbar_fence_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(&s_tmem, CT::T_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before_sync();
+  __syncthreads();
+  tc_fence_after_sync();
+  const uint32_t tmem = s_tmem;
+  const uint32_t lane_base = static_cast<uint32_t>(32 * (warp & 3)) << 16;
+  const uint32_t t_st = tmem + CT::T_ST + lane_base;
+  const uint32_t t_g1 = tmem + CT::T_G1 + lane_base;
+  const uint32_t t_gr = tmem + CT::T_GR + lane_base;
+  uint32_t phase = 0;
+  bool aborted = false;
+  // bounded wait for the last commit, decided by the whole CTA
+  auto wait_mma = [&]() -> bool {
+    const bool late = !mbar_wait(&bar, phase);
+    phase ^= 1u;
+    const bool any = __syncthreads_or(late) != 0;
+    tc_fence_after_sync();
+    return any;
+  };
+
+  const float expA = expf(p.A_log[hv]);
+  const float dtb = p.dt_bias[hv];
+  float na = 0.f, nb = 0.f;  // raw gate and beta of the next chunk (threads < C)
+  auto load_ab = [&](int64_t base) {
+    if (tid < C) {
+      const int64_t pos = base + tid;
+      if (pos >= pos_lo && pos < pos_hi) {
+        const int64_t tok = u.tok0 + (pos - pos_lo);
+        na = ld_in1(p.gate, tok * p.HV + hv, in_bf16);
+        nb = ld_in1(p.beta, tok * p.HV + hv, in_bf16);
+      }
+    }
+  };
+  chunk_issue_loads(p, sm, 0, base0, pos_lo, pos_hi, u.tok0, h, hv);
+  load_ab(base0);
+
+  for (int c = 0; c < nchunks && !aborted; ++c) {
+    const int buf = c & 1;
+    const int64_t base = base0 + (int64_t)c * C;
+    const float ca = na, cb = nb;
+    cp_async_wait_all();
+    __syncthreads();
+    if (c + 1 < nchunks) {
+      chunk_issue_loads(p, sm, buf ^ 1, base + C, pos_lo, pos_hi, u.tok0, h, hv);
+      load_ab(base + C);
+    }
+    const unsigned char* kq = sm + CT::KQ + buf * CT::KQ_BYTES;
+
+    // ---- per-token scalars: log alpha prefix (double), beta, norms
+    if (tid < C) {
+      const int64_t pos = base + tid;
+      const bool valid = pos >= pos_lo && pos < pos_hi;
+      const float la = valid ? -expA * softplus_f(ca + dtb) : 0.0f;
+      s_beta[tid] = valid ? ((p.flags & F_BETA_PROB) ? cb : sigmoid_f(cb)) : 0.0f;
+      double x = static_cast<double>(la);
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const double y = __shfl_up_sync(kFull, x, o);
+        if (lane >= o) x += y;
+      }
+      s_g[tid] = x;
+      if (tid == 31) s_wsum = x;
+    }
+    float ss = 0.f;  // row v of [K ; Q], this warpgroup's 64 columns
+#pragma unroll
+    for (int c8 = 0; c8 < D / 16; ++c8) {
+      const uint4 w = *reinterpret_cast<const uint4*>(kq + kmajor_offset(v, 64 * wg + 8 * c8, D));
+      const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float lo = bf16_lo(ww[e]), hi = bf16_hi(ww[e]);
+        ss = fmaf(lo, lo, ss);
+        ss = fmaf(hi, hi, ss);
+      }
+    }
+    if (wg == 1) s_nrm[v] = ss;
+    __syncthreads();
+    if (tid >= 32 && tid < C) s_g[tid] += s_wsum;
+    if (wg == 0) {
+      const float inv = (p.flags & F_L2NORM) ? rsqrtf(ss + s_nrm[v] + kL2Eps) : 1.0f;
+      if (v < C) s_ik[v] = inv;
+      else s_iq[v - C] = inv * p.scale;
+    }
+    __syncthreads();
+    const double gC = s_g[C - 1];
+    const float eC = expf(static_cast<float>(gC));
+    if (tid < C) {
+      const float eg = expf(static_cast<float>(s_g[tid]));
+      s_egk[tid] = eg * s_ik[tid];
+      s_egq[tid] = eg * s_iq[tid];
+      s_wc[tid] = s_ik[tid] * expf(static_cast<float>(gC - s_g[tid]));
+    }
+
+    // ---- the state: previous chunk's update done; snapshot, split, decay
+    // (this warpgroup's 64 columns of row v)
+    if (c > 0 && wait_mma()) {
+      aborted = true;
+      break;
+    }
+    {
+      int64_t snap = -1;
+      if (c > 0) {
+        const int64_t last = base - 1;  // last position of the previous chunk
+        if (last >= pos_lo) snap = suffix_snapshot_page(p, u, static_cast<int>(last - pos_lo));
+      }
+      if (snap >= p.num_slots) {
+        if (tid == 0) raise_err(p.err, E_PAGE_RANGE);
+        snap = -1;
+      }
+#pragma unroll 1
+      for (int kk = 0; kk < 2; ++kk) {
+        const int kc = 2 * wg + kk;
+        float x[32];
+        if (c == 0) {
+          if (u.fresh) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) x[i] = 0.0f;
+          } else {
+            const float4* src = reinterpret_cast<const float4*>(pool + (u.src * p.HV + hv) * head + (int64_t)v * D + 32 * kc);
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+              const float4 f = __ldcs(src + q);
+              x[4 * q] = f.x; x[4 * q + 1] = f.y; x[4 * q + 2] = f.z; x[4 * q + 3] = f.w;
+            }
+          }
+        } else {
+          tmem_ld32(t_st + 32 * kc, x);
+        }
+        if (snap >= 0) {
+          float4* dst = reinterpret_cast<float4*>(pool + (snap * p.HV + hv) * head + (int64_t)v * D + 32 * kc);
+#pragma unroll
+          for (int q = 0; q < 8; ++q) __stcs(dst + q, make_float4(x[4 * q], x[4 * q + 1], x[4 * q + 2], x[4 * q + 3]));
+        }
+#pragma unroll
+        for (int q8 = 0; q8 < 4; ++q8) {
+          float hh[8], mm[8], ll[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) split_bf16x3(x[8 * q8 + e], hh[e], mm[e], ll[e]);
+          const uint32_t off = kmajor_offset(v, 32 * kc + 8 * q8, D);
+          *reinterpret_cast<uint4*>(sm + CT::S3 + off) = pack_bf16x8(hh);
+          *reinterpret_cast<uint4*>(sm + CT::S3 + CT::S3_BYTES + off) = pack_bf16x8(mm);
+          *reinterpret_cast<uint4*>(sm + CT::S3 + 2 * CT::S3_BYTES + off) = pack_bf16x8(ll);
+        }
+#pragma unroll
+        for (int i = 0; i < 32; ++i) x[i] *= eC;
+        tmem_st32(t_st + 32 * kc, x);
+      }
+    }
+    fence_async_smem();
+    tc_fence_before_sync();
+    __syncthreads();
+
+    // ---- G1 = S0^T [K ; Q]^T and Gram = [K ; Q] K^T on the tensor cores
+    if (tid == 0) {
+      tc_fence_after_sync();
+      const uint32_t id_g1 = umma_idesc_bf16(128, 128), id_gr = umma_idesc_bf16(128, 64);
+#pragma unroll 1
+      for (int i = 0; i < 3; ++i)
+#pragma unroll 1
+        for (int ks = 0; ks < D / 16; ++ks)
+          umma_bf16(tmem + CT::T_G1, umma_desc_kmajor(sm + CT::S3 + i * CT::S3_BYTES + ks * 256, D),
+                    umma_desc_kmajor(kq + ks * 256, D), id_g1, i > 0 || ks > 0);
+#pragma unroll 1
+      for (int ks = 0; ks < D / 16; ++ks)
+        umma_bf16(tmem + CT::T_GR, umma_desc_kmajor(kq + ks * 256, D), umma_desc_kmajor(kq + ks * 256, D), id_gr, ks > 0);
+      umma_commit(&bar);
+    }
+    if (wait_mma()) {
+      aborted = true;
+      break;
+    }
+
+    // ---- A and P rows from the Gram: thread (wg, r) takes columns 32 wg ..
+    // 32 wg + 31 of row r (k row r < 64, q row r - 64)
+    {
+      float gr[32];
+      tmem_ld32(t_gr + 32 * wg, gr);
+      const int t = v & (C - 1);
+      const bool is_p = v >= C;
+      const double gt = s_g[t];
+      const float coef = is_p ? s_iq[t] : s_beta[t] * s_ik[t];
+      const int lim = is_p ? t + 1 : t;  // columns s < lim are kept
+      float* row = reinterpret_cast<float*>(sm + (is_p ? CT::PM : CT::AM)) + t * CT::AS + 32 * wg;
+#pragma unroll
+      for (int s4 = 0; s4 < 32; s4 += 4) {
+        float w[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int sx = 32 * wg + s4 + e;
+          w[e] = sx < lim ? coef * s_ik[sx] * __expf(static_cast<float>(gt - s_g[sx])) * gr[s4 + e] : 0.0f;
+        }
+        *reinterpret_cast<float4*>(row + s4) = make_float4(w[0], w[1], w[2], w[3]);
+      }
+    }
+    // ---- K^T for the update: thread (wg, k) gathers 32 tokens of column k
+#pragma unroll
+    for (int tt = 0; tt < 4; ++tt) {
+      const int t8 = 4 * wg + tt;
+      uint32_t w[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const uint32_t lo = *reinterpret_cast<const uint16_t*>(kq + kmajor_offset(8 * t8 + 2 * i, v, D));
+        const uint32_t hi = *reinterpret_cast<const uint16_t*>(kq + kmajor_offset(8 * t8 + 2 * i + 1, v, D));
+        w[i] = lo | (hi << 16);
+      }
+      *reinterpret_cast<uint4*>(sm + CT::KT + kmajor_offset(v, 8 * t8, C)) = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+    __syncthreads();  // A, P, K^T are in shared memory; the [K ; Q] tile is free
+    // U lives in the chunk's [K ; Q] buffer from here on: Us[t][v]
+    float* Us = reinterpret_cast<float*>(sm + CT::KQ + buf * CT::KQ_BYTES);
+    // ---- residuals R_t = beta_t (v_t - e^{g_t} k^_t S0), tokens 32 wg .. 32 wg + 31
+    {
+      const __nv_bfloat16* vcol = reinterpret_cast<const __nv_bfloat16*>(sm + CT::VB + buf * CT::V_BYTES) + v;
+      float x[32];
+      tmem_ld32(t_g1 + 32 * wg, x);
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        const int t = 32 * wg + i;
+        Us[t * D + v] = s_beta[t] * (__bfloat162float(vcol[t * D]) - s_egk[t] * x[i]);
+      }
+    }
+    __syncthreads();
+    // ---- (I + A) U = R in blocks of 8 tokens: each warpgroup takes 4 rows of
+    // the block for the part from earlier blocks; the triangle inside the
+    // block is finished by the first warpgroup, then by the second
+    {
+      const float* Am = reinterpret_cast<const float*>(sm + CT::AM);
+#pragma unroll 1
+      for (int b8 = 0; b8 < C / 8; ++b8) {
+        const int t0 = 8 * b8, r0 = t0 + 4 * wg;
+        float uu[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) uu[i] = Us[(r0 + i) * D + v];
+#pragma unroll 1
+        for (int s4 = 0; s4 < t0; s4 += 4) {
+          float us[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) us[e] = Us[(s4 + e) * D + v];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const float4 a = *reinterpret_cast<const float4*>(Am + (r0 + i) * CT::AS + s4);
+            uu[i] -= a.x * us[0] + a.y * us[1] + a.z * us[2] + a.w * us[3];
+          }
+        }
+        if (wg == 0) {
+#pragma unroll
+          for (int i = 1; i < 4; ++i)
+#pragma unroll
+            for (int j = 0; j < i; ++j) uu[i] = fmaf(-Am[(t0 + i) * CT::AS + t0 + j], uu[j], uu[i]);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) Us[(t0 + i) * D + v] = uu[i];
+        }
+        __syncthreads();
+        if (wg == 1) {
+          float lo[4];
+#pragma unroll
+          for (int j = 0; j < 4; ++j) lo[j] = Us[(t0 + j) * D + v];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+#pragma unroll
+            for (int j = 0; j < 4; ++j) uu[i] = fmaf(-Am[(r0 + i) * CT::AS + t0 + j], lo[j], uu[i]);
+#pragma unroll
+            for (int j = 0; j < i; ++j) uu[i] = fmaf(-Am[(r0 + i) * CT::AS + r0 + j], uu[j], uu[i]);
+          }
+#pragma unroll
+          for (int i = 0; i < 4; ++i) Us[(r0 + i) * D + v] = uu[i];
+        }
+        __syncthreads();
+      }
+    }
+    // ---- outputs o_t = e^{g_t} q^_t S0 + sum_{s<=t} P_ts U_s (P is zero above
+    // the diagonal); blocks {0, 1, 2, 3, 7} and {4, 5, 6} balance the two warpgroups
+    {
+      const float* Pm = reinterpret_cast<const float*>(sm + CT::PM);
+#pragma unroll 1
+      for (int bi = 0; bi < (wg == 0 ? 5 : 3); ++bi) {
+        const int b8 = (wg == 0) ? (bi < 4 ? bi : 7) : 4 + bi;
+        const int t0 = 8 * b8;
+        float oo[8];
+        tmem_ld8(t_g1 + C + t0, oo);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) oo[i] *= s_egq[t0 + i];
+#pragma unroll 1
+        for (int s4 = 0; s4 < t0 + 8; s4 += 4) {
+          float us[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) us[e] = Us[(s4 + e) * D + v];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const float4 w = *reinterpret_cast<const float4*>(Pm + (t0 + i) * CT::AS + s4);
+            oo[i] += w.x * us[0] + w.y * us[1] + w.z * us[2] + w.w * us[3];
+          }
+        }
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const int64_t pos = base + t0 + i;
+          if (pos >= pos_lo && pos < pos_hi)
+            st_out1(p.out, ((u.tok0 + (pos - pos_lo)) * p.HV + hv) * D + v, oo[i], out_bf16);
+        }
+      }
+    }
+    // ---- update operand (diag(w) U)^T, split in three bf16 terms (tokens 32 wg ..)
+#pragma unroll 1
+    for (int tt = 0; tt < 4; ++tt) {
+      const int t8 = 4 * wg + tt;
+      float hh[8], mm[8], ll[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int t = 8 * t8 + i;
+        split_bf16x3(s_wc[t] * Us[t * D + v], hh[i], mm[i], ll[i]);
+      }
+      const uint32_t off = kmajor_offset(v, 8 * t8, C);
+      *reinterpret_cast<uint4*>(sm + CT::UT3 + off) = pack_bf16x8(hh);
+      *reinterpret_cast<uint4*>(sm + CT::UT3 + CT::UT_BYTES + off) = pack_bf16x8(mm);
+      *reinterpret_cast<uint4*>(sm + CT::UT3 + 2 * CT::UT_BYTES + off) = pack_bf16x8(ll);
+    }
+    fence_async_smem();
+    tc_fence_before_sync();
+    __syncthreads();
+    // ---- S^T += (diag(w) U)^T K on the tensor cores (the state was decayed above)
+    if (tid == 0) {
+      tc_fence_after_sync();
+      const uint32_t id_up = umma_idesc_bf16(128, 128);
+#pragma unroll 1
+      for (int i = 0; i < 3; ++i)
+#pragma unroll 1
+        for (int ks = 0; ks < C / 16; ++ks)
+          umma_bf16(tmem + CT::T_ST, umma_desc_kmajor(sm + CT::UT3 + i * CT::UT_BYTES + ks * 256, C),
+                    umma_desc_kmajor(sm + CT::KT + ks * 256, C), id_up, true);
+      umma_commit(&bar);
+    }
+  }
+
+  // ---- the final state to the last page (this warpgroup's 64 columns of row v)
+  if (!aborted) {
+    if (wait_mma()) {
+      aborted = true;
+    } else {
+      float4* dst = reinterpret_cast<float4*>(pool + (u.dst * p.HV + hv) * head + (int64_t)v * D);
+#pragma unroll 1
+      for (int kk = 0; kk < 2; ++kk) {
+        const int kc = 2 * wg + kk;
+        float x[32];
+        tmem_ld32(t_st + 32 * kc, x);
+#pragma unroll
+        for (int q = 0; q < 8; ++q) __stcs(dst + 8 * kc + q, make_float4(x[4 * q], x[4 * q + 1], x[4 * q + 2], x[4 * q + 3]));
+      }
+    }
+  }
+  if (aborted) {
+    if (tid == 0) raise_err(p.err, E_TIMEOUT);
+    (void)mbar_wait(&bar, phase ^ 1u);  // a bounded chance for the MMAs in flight to finish
+  }
+  cp_async_wait_all();
+  tc_fence_before_sync();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after_sync();
+    tmem_dealloc(tmem, CT::T_COLS);
+  }
+}
+
+}  // namespace gdn

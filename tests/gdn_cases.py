@@ -295,16 +295,30 @@ def gdn_paged_case(seed, B, H, HV, K, V, page_size, max_len, n_share, share_page
 # ----------------------------------------------------------------------------
 
 def gdn_prefill_case(seed, B, H, HV, K, V, page_size, max_len, state_dtype="f32", in_dtype="bf16",
-                     out_dtype="f32", index_dtype="i32", layout="V_FIRST", fresh_every=2):
-    pt = W.paged_table(seed, B, page_size, max_len, 0, 0).cast(index_dtype)
-    cu = W.prefill_runs(seed, pt.seq_lens.tolist(), fresh_every)
+                     out_dtype="f32", index_dtype="i32", layout="V_FIRST", fresh_every=2, scale=None,
+                     use_qk_l2norm=True, units=None, cu=None, min_len=2):
+    """One paged prefill on the GPU against the oracle. ``units`` restricts the
+    oracle (and the comparison) to some (sequence, value head) pairs; the
+    pages that must stay untouched are still checked for every sequence."""
+    pt = W.paged_table(seed, B, page_size, max_len, 0, 0, min_len=min_len).cast(index_dtype)
+    cu = np.asarray(cu if cu is not None else W.prefill_runs(seed, pt.seq_lens.tolist(), fresh_every), np.int32)
     total = int(cu[-1])
     t = W.varlen_gdn_tokens(seed, total, H, HV, K, V, in_dtype)
-    reads = set()
+    reads, written = set(), set()
     for bb in range(B):
         n = int(cu[bb + 1] - cu[bb])
-        if 0 < n < int(pt.seq_lens[bb]):
-            reads.add(O.suffix_pages(pt.page_indices, pt.page_indptr, pt.last_page_len, page_size, n, bb)[0])
+        if n == 0:
+            continue
+        L = int(pt.seq_lens[bb])
+        if n < L:
+            rd, snaps, last = O.suffix_pages(pt.page_indices, pt.page_indptr, pt.last_page_len, page_size, n, bb)
+            reads.add(rd)
+            written.update(pg for _, pg in snaps)
+        else:  # a fresh sequence fills every page it owns
+            p0 = int(pt.page_indptr[bb])
+            written.update(int(pt.page_indices[p0 + i]) for i in range((L - 1) // page_size))
+            last = int(pt.page_indices[int(pt.page_indptr[bb + 1]) - 1])
+        written.add(last)
     pool, scales = W.device_pool(seed, pt.num_pages, HV, K, V, layout, state_dtype, exact_slots=sorted(reads))
     snap = pool.clone()
     sc_snap = scales.clone() if scales is not None else None
@@ -314,18 +328,20 @@ def gdn_prefill_case(seed, B, H, HV, K, V, page_size, max_len, state_dtype="f32"
         dev_in(t["b"], in_dtype), dev(t["A_log"]), dev(t["dt_bias"]), dev(cu), state_pool=pool,
         page_indices=dev(pt.page_indices), page_indptr=dev(pt.page_indptr), last_page_len=dev(pt.last_page_len),
         page_size=page_size, state_scales=scales, state_layout=layout, output_dtype=W.torch_dtype(out_dtype),
-        err_flags=err)
+        scale=scale, use_qk_l2norm=use_qk_l2norm, err_flags=err)
     torch.cuda.synchronize()
     states, sc = W.host_pool(seed, sorted(reads), HV, K, V, layout, state_dtype)
     ref_out, writes = O.gdn_prefill_paged(t["q"], t["k"], t["v"], t["a"], t["b"], t["A_log"], t["dt_bias"], cu,
                                           states, pt.page_indices, pt.page_indptr, pt.last_page_len, page_size,
-                                          state_dtype=state_dtype, state_scales=sc, layout=layout)
-    units = [(bb, hv) for bb in range(B) for hv in range(HV)]
+                                          state_dtype=state_dtype, state_scales=sc, layout=layout, scale=scale,
+                                          use_qk_l2norm=use_qk_l2norm, units=units)
+    todo = [(bb, hv) for bb in range(B) for hv in range(HV)] if units is None else list(units)
     res = dict(err=int(err.item()), cu=cu, table=pt)
-    res["out_err"] = check_outputs(host(out), ref_out, units, lambda x, bb, hv: x[int(cu[bb]):int(cu[bb + 1]), hv, :],
+    res["out_err"] = check_outputs(host(out), ref_out, todo, lambda x, bb, hv: x[int(cu[bb]):int(cu[bb + 1]), hv, :],
                                    out_tol(state_dtype, "working", True), out_dtype)
-    write_pages = sorted({pg for (pg, _) in writes})
-    wp = torch.tensor(write_pages, device="cuda")
+    write_pages = sorted(written)
+    assert {pg for (pg, _) in writes} <= set(write_pages)
+    wp = torch.tensor(write_pages, device="cuda", dtype=torch.long)
     pos = {pg: i for i, pg in enumerate(write_pages)}
     res["state_err"] = check_state(pool_host(pool[wp]), scales[wp].cpu().numpy() if scales is not None else None,
                                    {(pos[pg], hv): w for (pg, hv), w in writes.items()}, state_dtype, layout)
