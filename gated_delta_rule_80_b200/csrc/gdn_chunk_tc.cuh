@@ -47,14 +47,18 @@ struct ChunkTC {
   static constexpr uint32_t V_BYTES = C * D * 2;
   static constexpr uint32_t S3 = VB + 2 * V_BYTES;  // 3 x [128 x 128] bf16, K-major: S0^T split
   static constexpr uint32_t S3_BYTES = D * D * 2;
-  // after G1 the S3 region holds the chunk's update operands and A, P
-  static constexpr uint32_t UT3 = S3;                 // 3 x [128 x 64] bf16, K-major: (diag(w) U)^T split
+  // after G1 the S3 region holds A (fp32, for the solve), then in its place
+  // U^T and later (diag(w) U)^T (three bf16 terms each), K^T, and P (three
+  // bf16 terms)
+  static constexpr uint32_t UT3 = S3;                 // 3 x [128 x 64] bf16, K-major
   static constexpr uint32_t UT_BYTES = D * C * 2;
+  static constexpr int AS = C + 4;                    // row stride of A (floats), staggers banks
+  static constexpr uint32_t AM = S3;                  // [64 x AS] fp32, inside the UT3 area
   static constexpr uint32_t KT = UT3 + 3 * UT_BYTES;  // [128 x 64] bf16, K-major: K^T
-  static constexpr int AS = C + 4;                    // row stride of A and P (floats), staggers banks
-  static constexpr uint32_t AM = KT + UT_BYTES;       // [64 x AS] fp32
-  static constexpr uint32_t PM = AM + C * AS * 4;     // [64 x AS] fp32
-  static constexpr uint32_t SMEM = (PM + C * AS * 4 > S3 + 3 * S3_BYTES) ? PM + C * AS * 4 : S3 + 3 * S3_BYTES;
+  static constexpr uint32_t P3 = KT + UT_BYTES;       // 3 x [64 x 64] bf16, K-major: P split
+  static constexpr uint32_t P_BYTES = C * C * 2;
+  static constexpr uint32_t SMEM = S3 + 3 * S3_BYTES;
+  static_assert(AM + C * AS * 4 <= KT && P3 + 3 * P_BYTES <= SMEM, "chunk operands fit in the S3 region");
   // tensor memory columns
   static constexpr uint32_t T_ST = 0, T_G1 = 128, T_GR = 256, T_COLS = 512;
 };
@@ -122,12 +126,15 @@ __global__ void __launch_bounds__(ChunkTC::NT, 1) prefill_chunk_tc(const StepPar
   using CT = ChunkTC;
   constexpr int C = CT::C, D = CT::D;
   extern __shared__ __align__(1024) unsigned char sm[];
-  __shared__ __align__(8) uint64_t bar;
+  // MMA completion: one barrier for the Gram, one for G1 and the update, so
+  // that neither ever has more than one phase outstanding
+  __shared__ __align__(8) uint64_t bar, bar_gr;
   __shared__ uint32_t s_tmem;
   __shared__ double s_g[C];
   __shared__ double s_wsum;
   __shared__ float s_beta[C], s_ik[C], s_iq[C];
   __shared__ float s_egk[C], s_egq[C], s_wc[C];  // e^{g_t} |k_t|^-1, e^{g_t} scale |q_t|^-1, |k_t|^-1 e^{g_C - g_t}
+  __shared__ float s_eg[C], s_kinv[C];           // e^{g_t}; |k_t|^-1 e^{-g_t} (chunks with g_C > -80)
   __shared__ float s_nrm[D];                     // the second warpgroup's half of each row's sum of squares
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -155,6 +162,7 @@ __global__ void __launch_bounds__(ChunkTC::NT, 1) prefill_chunk_tc(const StepPar
 
   if (tid == 0) {
     mbar_init(&bar, 1);
+    mbar_init(&bar_gr, 1);
     mbar_fence_init();
   }
   if (warp == 0) {
@@ -169,16 +177,17 @@ __global__ void __launch_bounds__(ChunkTC::NT, 1) prefill_chunk_tc(const StepPar
   const uint32_t t_st = tmem + CT::T_ST + lane_base;
   const uint32_t t_g1 = tmem + CT::T_G1 + lane_base;
   const uint32_t t_gr = tmem + CT::T_GR + lane_base;
-  uint32_t phase = 0;
+  uint32_t phase = 0, phase_gr = 0;
   bool aborted = false;
-  // bounded wait for the last commit, decided by the whole CTA
-  auto wait_mma = [&]() -> bool {
-    const bool late = !mbar_wait(&bar, phase);
-    phase ^= 1u;
+  // bounded wait for the oldest commit on `bar` (or on `bar_gr`), decided by the whole CTA
+  auto wait_on = [&](uint64_t* br, uint32_t& ph) -> bool {
+    const bool late = !mbar_wait(br, ph);
+    ph ^= 1u;
     const bool any = __syncthreads_or(late) != 0;
     tc_fence_after_sync();
     return any;
   };
+  auto wait_mma = [&]() -> bool { return wait_on(&bar, phase); };
 
   const float expA = expf(p.A_log[hv]);
   const float dtb = p.dt_bias[hv];
@@ -247,7 +256,9 @@ __global__ void __launch_bounds__(ChunkTC::NT, 1) prefill_chunk_tc(const StepPar
     const double gC = s_g[C - 1];
     const float eC = expf(static_cast<float>(gC));
     if (tid < C) {
-      const float eg = expf(static_cast<float>(s_g[tid]));
+      const float eg = static_cast<float>(exp(s_g[tid]));  // double: the exponent is not rounded to fp32 first
+      s_eg[tid] = eg;
+      s_kinv[tid] = gC > -80.0 ? s_ik[tid] * static_cast<float>(exp(-s_g[tid])) : 0.0f;
       s_egk[tid] = eg * s_ik[tid];
       s_egq[tid] = eg * s_iq[tid];
       s_wc[tid] = s_ik[tid] * expf(static_cast<float>(gC - s_g[tid]));
@@ -317,23 +328,26 @@ __global__ void __launch_bounds__(ChunkTC::NT, 1) prefill_chunk_tc(const StepPar
       tc_fence_after_sync();
       const uint32_t id_g1 = umma_idesc_bf16(128, 128), id_gr = umma_idesc_bf16(128, 64);
 #pragma unroll 1
+      for (int ks = 0; ks < D / 16; ++ks)
+        umma_bf16(tmem + CT::T_GR, umma_desc_kmajor(kq + ks * 256, D), umma_desc_kmajor(kq + ks * 256, D), id_gr, ks > 0);
+      umma_commit(&bar_gr);
+#pragma unroll 1
       for (int i = 0; i < 3; ++i)
 #pragma unroll 1
         for (int ks = 0; ks < D / 16; ++ks)
           umma_bf16(tmem + CT::T_G1, umma_desc_kmajor(sm + CT::S3 + i * CT::S3_BYTES + ks * 256, D),
                     umma_desc_kmajor(kq + ks * 256, D), id_g1, i > 0 || ks > 0);
-#pragma unroll 1
-      for (int ks = 0; ks < D / 16; ++ks)
-        umma_bf16(tmem + CT::T_GR, umma_desc_kmajor(kq + ks * 256, D), umma_desc_kmajor(kq + ks * 256, D), id_gr, ks > 0);
       umma_commit(&bar);
     }
-    if (wait_mma()) {
+    // the Gram first: A, P and K^T do not wait for G1
+    if (wait_on(&bar_gr, phase_gr)) {
       aborted = true;
       break;
     }
 
     // ---- A and P rows from the Gram: thread (wg, r) takes columns 32 wg ..
-    // 32 wg + 31 of row r (k row r < 64, q row r - 64)
+    // 32 wg + 31 of row r (k row r < 64: A in fp32; q row r - 64: P as three
+    // bf16 tiles, the B operand of the output product)
     {
       float gr[32];
       tmem_ld32(t_gr + 32 * wg, gr);
@@ -342,16 +356,31 @@ __global__ void __launch_bounds__(ChunkTC::NT, 1) prefill_chunk_tc(const StepPar
       const double gt = s_g[t];
       const float coef = is_p ? s_iq[t] : s_beta[t] * s_ik[t];
       const int lim = is_p ? t + 1 : t;  // columns s < lim are kept
-      float* row = reinterpret_cast<float*>(sm + (is_p ? CT::PM : CT::AM)) + t * CT::AS + 32 * wg;
+      // e^{g_t - g_s} = e^{g_t} e^{-g_s} while e^{-g_C} stays finite; per pair otherwise
+      const bool factored = gC > -80.0;
+      const float ct = coef * (factored ? s_eg[t] : 1.0f);
+      float* arow = reinterpret_cast<float*>(sm + CT::AM) + t * CT::AS + 32 * wg;
 #pragma unroll
-      for (int s4 = 0; s4 < 32; s4 += 4) {
-        float w[4];
+      for (int s8 = 0; s8 < 32; s8 += 8) {
+        float w[8];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int sx = 32 * wg + s4 + e;
-          w[e] = sx < lim ? coef * s_ik[sx] * __expf(static_cast<float>(gt - s_g[sx])) * gr[s4 + e] : 0.0f;
+        for (int e = 0; e < 8; ++e) {
+          const int sx = 32 * wg + s8 + e;
+          const float d = factored ? s_kinv[sx] : s_ik[sx] * __expf(static_cast<float>(gt - s_g[sx]));
+          w[e] = sx < lim ? ct * d * gr[s8 + e] : 0.0f;
         }
-        *reinterpret_cast<float4*>(row + s4) = make_float4(w[0], w[1], w[2], w[3]);
+        if (is_p) {
+          float hh[8], mm[8], ll[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) split_bf16x3(w[e], hh[e], mm[e], ll[e]);
+          const uint32_t off = kmajor_offset(t, 32 * wg + s8, C);
+          *reinterpret_cast<uint4*>(sm + CT::P3 + off) = pack_bf16x8(hh);
+          *reinterpret_cast<uint4*>(sm + CT::P3 + CT::P_BYTES + off) = pack_bf16x8(mm);
+          *reinterpret_cast<uint4*>(sm + CT::P3 + 2 * CT::P_BYTES + off) = pack_bf16x8(ll);
+        } else {
+          *reinterpret_cast<float4*>(arow + s8) = make_float4(w[0], w[1], w[2], w[3]);
+          *reinterpret_cast<float4*>(arow + s8 + 4) = make_float4(w[4], w[5], w[6], w[7]);
+        }
       }
     }
     // ---- K^T for the update: thread (wg, k) gathers 32 tokens of column k
@@ -367,7 +396,10 @@ __global__ void __launch_bounds__(ChunkTC::NT, 1) prefill_chunk_tc(const StepPar
       }
       *reinterpret_cast<uint4*>(sm + CT::KT + kmajor_offset(v, 8 * t8, C)) = make_uint4(w[0], w[1], w[2], w[3]);
     }
-    __syncthreads();  // A, P, K^T are in shared memory; the [K ; Q] tile is free
+    if (wait_mma()) {  // G1; also orders A, P and K^T before the reads below
+      aborted = true;
+      break;
+    }
     // U lives in the chunk's [K ; Q] buffer from here on: Us[t][v]
     float* Us = reinterpret_cast<float*>(sm + CT::KQ + buf * CT::KQ_BYTES);
     // ---- residuals R_t = beta_t (v_t - e^{g_t} k^_t S0), tokens 32 wg .. 32 wg + 31
@@ -382,83 +414,113 @@ __global__ void __launch_bounds__(ChunkTC::NT, 1) prefill_chunk_tc(const StepPar
       }
     }
     __syncthreads();
-    // ---- (I + A) U = R in blocks of 8 tokens: each warpgroup takes 4 rows of
-    // the block for the part from earlier blocks; the triangle inside the
-    // block is finished by the first warpgroup, then by the second
+    // ---- (I + A) U = R in two blocks of 32 tokens: each warpgroup takes 16
+    // rows of the block for the part from the earlier block; the triangle
+    // inside the block is finished by the first warpgroup, then by the second
     {
+      constexpr int BS = 32, HB = BS / 2;
       const float* Am = reinterpret_cast<const float*>(sm + CT::AM);
 #pragma unroll 1
-      for (int b8 = 0; b8 < C / 8; ++b8) {
-        const int t0 = 8 * b8, r0 = t0 + 4 * wg;
-        float uu[4];
+      for (int bb = 0; bb < C / BS; ++bb) {
+        const int t0 = BS * bb, r0 = t0 + HB * wg;
+        float uu[HB];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) uu[i] = Us[(r0 + i) * D + v];
+        for (int i = 0; i < HB; ++i) uu[i] = Us[(r0 + i) * D + v];
 #pragma unroll 1
         for (int s4 = 0; s4 < t0; s4 += 4) {
           float us[4];
 #pragma unroll
           for (int e = 0; e < 4; ++e) us[e] = Us[(s4 + e) * D + v];
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
+          for (int i = 0; i < HB; ++i) {
             const float4 a = *reinterpret_cast<const float4*>(Am + (r0 + i) * CT::AS + s4);
-            uu[i] -= a.x * us[0] + a.y * us[1] + a.z * us[2] + a.w * us[3];
+            uu[i] = fmaf(-a.x, us[0], uu[i]);
+            uu[i] = fmaf(-a.y, us[1], uu[i]);
+            uu[i] = fmaf(-a.z, us[2], uu[i]);
+            uu[i] = fmaf(-a.w, us[3], uu[i]);
           }
         }
         if (wg == 0) {
 #pragma unroll
-          for (int i = 1; i < 4; ++i)
+          for (int i = 1; i < HB; ++i)
 #pragma unroll
             for (int j = 0; j < i; ++j) uu[i] = fmaf(-Am[(t0 + i) * CT::AS + t0 + j], uu[j], uu[i]);
 #pragma unroll
-          for (int i = 0; i < 4; ++i) Us[(t0 + i) * D + v] = uu[i];
+          for (int i = 0; i < HB; ++i) Us[(t0 + i) * D + v] = uu[i];
         }
         __syncthreads();
         if (wg == 1) {
-          float lo[4];
 #pragma unroll
-          for (int j = 0; j < 4; ++j) lo[j] = Us[(t0 + j) * D + v];
+          for (int j4 = 0; j4 < HB; j4 += 4) {
+            float lo[4];
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
+            for (int e = 0; e < 4; ++e) lo[e] = Us[(t0 + j4 + e) * D + v];
 #pragma unroll
-            for (int j = 0; j < 4; ++j) uu[i] = fmaf(-Am[(r0 + i) * CT::AS + t0 + j], lo[j], uu[i]);
-#pragma unroll
-            for (int j = 0; j < i; ++j) uu[i] = fmaf(-Am[(r0 + i) * CT::AS + r0 + j], uu[j], uu[i]);
+            for (int i = 0; i < HB; ++i) {
+              const float4 a = *reinterpret_cast<const float4*>(Am + (r0 + i) * CT::AS + t0 + j4);
+              uu[i] = fmaf(-a.x, lo[0], uu[i]);
+              uu[i] = fmaf(-a.y, lo[1], uu[i]);
+              uu[i] = fmaf(-a.z, lo[2], uu[i]);
+              uu[i] = fmaf(-a.w, lo[3], uu[i]);
+            }
           }
 #pragma unroll
-          for (int i = 0; i < 4; ++i) Us[(r0 + i) * D + v] = uu[i];
+          for (int i = 1; i < HB; ++i)
+#pragma unroll
+            for (int j = 0; j < i; ++j) uu[i] = fmaf(-Am[(r0 + i) * CT::AS + r0 + j], uu[j], uu[i]);
+#pragma unroll
+          for (int i = 0; i < HB; ++i) Us[(r0 + i) * D + v] = uu[i];
         }
         __syncthreads();
       }
     }
-    // ---- outputs o_t = e^{g_t} q^_t S0 + sum_{s<=t} P_ts U_s (P is zero above
-    // the diagonal); blocks {0, 1, 2, 3, 7} and {4, 5, 6} balance the two warpgroups
-    {
-      const float* Pm = reinterpret_cast<const float*>(sm + CT::PM);
+    // ---- outputs o_t = e^{g_t} q^_t S0 + sum_{s<=t} P_ts U_s: U^T (three bf16
+    // terms, replacing A) times P^T on the tensor cores (the six products of
+    // the splits above the lowest order), then the state part added
 #pragma unroll 1
-      for (int bi = 0; bi < (wg == 0 ? 5 : 3); ++bi) {
-        const int b8 = (wg == 0) ? (bi < 4 ? bi : 7) : 4 + bi;
-        const int t0 = 8 * b8;
-        float oo[8];
-        tmem_ld8(t_g1 + C + t0, oo);
+    for (int tt = 0; tt < 4; ++tt) {
+      const int t8 = 4 * wg + tt;
+      float hh[8], mm[8], ll[8];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) oo[i] *= s_egq[t0 + i];
+      for (int i = 0; i < 8; ++i) split_bf16x3(Us[(8 * t8 + i) * D + v], hh[i], mm[i], ll[i]);
+      const uint32_t off = kmajor_offset(v, 8 * t8, C);
+      *reinterpret_cast<uint4*>(sm + CT::UT3 + off) = pack_bf16x8(hh);
+      *reinterpret_cast<uint4*>(sm + CT::UT3 + CT::UT_BYTES + off) = pack_bf16x8(mm);
+      *reinterpret_cast<uint4*>(sm + CT::UT3 + 2 * CT::UT_BYTES + off) = pack_bf16x8(ll);
+    }
+    fence_async_smem();
+    tc_fence_before_sync();
+    __syncthreads();
+    if (tid == 0) {
+      tc_fence_after_sync();
+      const uint32_t id_o = umma_idesc_bf16(128, 64);
+      bool acc = false;
 #pragma unroll 1
-        for (int s4 = 0; s4 < t0 + 8; s4 += 4) {
-          float us[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) us[e] = Us[(s4 + e) * D + v];
-#pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            const float4 w = *reinterpret_cast<const float4*>(Pm + (t0 + i) * CT::AS + s4);
-            oo[i] += w.x * us[0] + w.y * us[1] + w.z * us[2] + w.w * us[3];
+      for (int i = 0; i < 3; ++i)
+#pragma unroll 1
+        for (int j = 0; i + j < 3; ++j)
+#pragma unroll 1
+          for (int ks = 0; ks < C / 16; ++ks) {
+            umma_bf16(tmem + CT::T_GR, umma_desc_kmajor(sm + CT::UT3 + i * CT::UT_BYTES + ks * 256, C),
+                      umma_desc_kmajor(sm + CT::P3 + j * CT::P_BYTES + ks * 256, C), id_o, acc);
+            acc = true;
           }
-        }
+      umma_commit(&bar_gr);
+    }
+    if (wait_on(&bar_gr, phase_gr)) {
+      aborted = true;
+      break;
+    }
+    {
+      float pu[32], ob[32];
+      tmem_ld32(t_gr + 32 * wg, pu);
+      tmem_ld32(t_g1 + C + 32 * wg, ob);
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const int64_t pos = base + t0 + i;
-          if (pos >= pos_lo && pos < pos_hi)
-            st_out1(p.out, ((u.tok0 + (pos - pos_lo)) * p.HV + hv) * D + v, oo[i], out_bf16);
-        }
+      for (int i = 0; i < 32; ++i) {
+        const int t = 32 * wg + i;
+        const int64_t pos = base + t;
+        if (pos >= pos_lo && pos < pos_hi)
+          st_out1(p.out, ((u.tok0 + (pos - pos_lo)) * p.HV + hv) * D + v, fmaf(s_egq[t], ob[i], pu[i]), out_bf16);
       }
     }
     // ---- update operand (diag(w) U)^T, split in three bf16 terms (tokens 32 wg ..)
@@ -511,7 +573,10 @@ __global__ void __launch_bounds__(ChunkTC::NT, 1) prefill_chunk_tc(const StepPar
   }
   if (aborted) {
     if (tid == 0) raise_err(p.err, E_TIMEOUT);
-    (void)mbar_wait(&bar, phase ^ 1u);  // a bounded chance for the MMAs in flight to finish
+    // a bounded chance for the MMAs in flight to finish (the last commit on
+    // each barrier; an already completed phase returns at once)
+    (void)mbar_wait(&bar, phase ^ 1u);
+    (void)mbar_wait(&bar_gr, phase_gr ^ 1u);
   }
   cp_async_wait_all();
   tc_fence_before_sync();
