@@ -35,22 +35,6 @@ __device__ __forceinline__ uint64_t umma_desc_kmajor(const void* tile, uint32_t 
          (1ull << 46);
 }
 
-// The same tile in the 128-byte swizzled K-major layout: 8-row x 64-column
-// atoms of 1 KiB (each row 128 contiguous bytes, its 16-byte chunks permuted
-// by XOR with the row index within the atom), atoms stacked along the rows
-// (SBO = 1 KiB) and, for more than 64 columns, whole column blocks of
-// R * 128 bytes after one another. Tiles start on 1 KiB boundaries.
-__host__ __device__ constexpr uint32_t sw128_offset(uint32_t r, uint32_t c, uint32_t R) {
-  return (c >> 6) * (R * 128u) + (r >> 3) * 1024u + (r & 7u) * 128u + ((((c & 63u) >> 3) ^ (r & 7u)) << 4) +
-         (c & 7u) * 2u;
-}
-// Descriptor of the 16 columns c0 .. c0 + 15 (c0 a multiple of 16) of such a
-// tile of R rows: SBO = 1 KiB, LBO unused (1), layout type 2 (128-byte swizzle).
-__device__ __forceinline__ uint64_t umma_desc_sw128(const void* tile, uint32_t c0, uint32_t R) {
-  const uint64_t addr = smem_addr(tile) + (c0 >> 6) * (R * 128u) + ((c0 & 63u) >> 3) * 16u;
-  return ((addr >> 4) & 0x3FFFull) | (1ull << 16) | ((1024ull >> 4) << 32) | (1ull << 46) | (2ull << 61);
-}
-
 // Instruction descriptor of kind::f16 with bf16 A and B (both K-major) and
 // an fp32 accumulator: c_format F32 in [4,6), a_format BF16 in [7,10),
 // b_format BF16 in [10,13), N >> 3 in [17,23), M >> 4 in [24,29).
