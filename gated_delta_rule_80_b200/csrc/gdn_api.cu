@@ -92,12 +92,10 @@ int launch_tile1(StepParams p, int B, cudaStream_t s) {
   return launch_status();
 }
 
-// Single-token GDN decode on a V_FIRST int8_hadamard32 pool: persistent
-// CTAs (as many as fit on the device at once) over the (sequence, value head,
-// scale group) tiles.
-template <int K, int IDX>
-int launch_pipe_i8(StepParams p, int B, cudaStream_t s) {
-  using PS = PipeI8Shape<K>;
+// Single-token GDN decode on a V_FIRST int8_hadamard32 pool: persistent CTAs (as many as fit on the device at once) over the (sequence,
+// value head, tile) units.
+template <class PS, class Kernel>
+int launch_pipe(Kernel kernel, StepParams p, int B, cudaStream_t s) {
   static int resident[64] = {0};  // CTAs per SM, per device
   int dev = 0, sms = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64 ||
@@ -107,10 +105,8 @@ int launch_pipe_i8(StepParams p, int B, cudaStream_t s) {
   }
   if (resident[dev] == 0) {
     int n = 0;
-    if (cudaFuncSetAttribute(step_pipe_i8<K, IDX>, cudaFuncAttributeMaxDynamicSharedMemorySize, PS::SMEM) !=
-            cudaSuccess ||
-        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, step_pipe_i8<K, IDX>, PS::NT, PS::SMEM) != cudaSuccess ||
-        n < 1) {
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, PS::SMEM) != cudaSuccess ||
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel, PS::NT, PS::SMEM) != cudaSuccess || n < 1) {
       cudaGetLastError();
       return GDN_ERR_CUDA;
     }
@@ -118,7 +114,7 @@ int launch_pipe_i8(StepParams p, int B, cudaStream_t s) {
   }
   const int64_t n_tiles = (int64_t)B * p.HV * (p.V / PS::VT);
   const int64_t grid = std::min<int64_t>(n_tiles, (int64_t)sms * resident[dev]);
-  step_pipe_i8<K, IDX><<<static_cast<unsigned>(grid), PS::NT, PS::SMEM, s>>>(p, n_tiles);
+  kernel<<<static_cast<unsigned>(grid), PS::NT, PS::SMEM, s>>>(p, n_tiles);
   return launch_status();
 }
 
@@ -162,7 +158,7 @@ int launch_one(StepParams p, int B, cudaStream_t s) {
   constexpr bool CODED = (SDT == ST_FP8 || SDT == ST_I8H);
   if constexpr (L == L_VFIRST && GATE == GATE_SCALAR) {
     if (p.T == 1) {
-      if constexpr (SDT == ST_I8H) return launch_pipe_i8<K, IDX>(p, B, s);
+      if constexpr (SDT == ST_I8H) return launch_pipe<PipeI8Shape<K>>(step_pipe_i8<K, IDX>, p, B, s);
       else return launch_tile1<SDT, K, IDX>(p, B, s);
     }
   }
