@@ -92,8 +92,9 @@ int launch_tile1(StepParams p, int B, cudaStream_t s) {
   return launch_status();
 }
 
-// Single-token GDN decode on a V_FIRST int8_hadamard32 pool: persistent CTAs (as many as fit on the device at once) over the (sequence,
-// value head, tile) units.
+// Single-token GDN decode on a V_FIRST int8_hadamard32 pool: persistent CTAs
+// (as many as fit on the device at once) over the (sequence, value head,
+// tile) units.
 template <class PS, class Kernel>
 int launch_pipe(Kernel kernel, StepParams p, int B, cudaStream_t s) {
   static int resident[64] = {0};  // CTAs per SM, per device
