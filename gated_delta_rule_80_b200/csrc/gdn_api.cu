@@ -87,6 +87,12 @@ template <int SDT, int K, int IDX>
 int launch_tile1(StepParams p, int B, cudaStream_t s) {
   using TS = Tile1Shape<SDT, K>;
   p.n_vtiles = p.V / TS::VT;
+  if constexpr (SDT == ST_FP8) {  // two tiles per CTA where the head has an even number
+    if (p.n_vtiles % 2 == 0) {
+      step_tile1<SDT, K, IDX, 2><<<dim3(p.n_vtiles / 2, p.HV, B), TS::NW * 32, 0, s>>>(p);
+      return launch_status();
+    }
+  }
   const dim3 grid(p.n_vtiles, p.HV, B);
   step_tile1<SDT, K, IDX><<<grid, TS::NW * 32, 0, s>>>(p);
   return launch_status();

@@ -111,8 +111,12 @@ struct ReduceScatter {
   }
 };
 
-template <int SDT, int K, int IDX>
-__global__ void __launch_bounds__(Tile1Shape<SDT, K>::NW * 32, Tile1Shape<SDT, K>::MIN_CTAS)
+// TPC consecutive tiles of one (sequence, value head) per CTA: every state
+// load of all of them is issued before the first is computed, and the token
+// prologue is shared (fp8 uses 2: twice the bytes in flight per thread for
+// 16 more registers).
+template <int SDT, int K, int IDX, int TPC = 1>
+__global__ void __launch_bounds__(Tile1Shape<SDT, K>::NW * 32, (TPC == 1 ? Tile1Shape<SDT, K>::MIN_CTAS : 3))
 step_tile1(const StepParams p) {
   using ST = StateTraits<SDT>;
   using TS = Tile1Shape<SDT, K>;
@@ -131,7 +135,7 @@ step_tile1(const StepParams p) {
   constexpr int ROWB = K * ST::BYTES;  // bytes of one stored row
 
   __shared__ float s_pro[5];           // alpha, beta, q scale, k scale, q^.k^
-  __shared__ float s_amax[NW];
+  __shared__ float s_amax[TPC][NW];
 
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
@@ -142,41 +146,49 @@ step_tile1(const StepParams p) {
   const bool holds_q = (vidx & 1) != 0;
   const int grp = lane - li;
   const bool writer = !holds_q && (li % REP) == 0;
-  const int tile = blockIdx.x;
+  const int tile0 = blockIdx.x * TPC;
   const int hv = blockIdx.y;
   const int b = blockIdx.z;            // T == 1: the token of sequence b is b
   const int h = hv / p.G;
   const int kofs = li * EPL;
   const bool in_bf16 = (p.flags & F_IN_BF16) != 0;
-  const int row0 = tile * VT + warp * NR * RPW + ri;   // row jj is row0 + jj * RPW
-  const int myrow_v = row0 + myrow * RPW;
+  const int row0r = warp * NR * RPW + ri;   // tile row of row jj: row0r + jj * RPW
 
   const Unit u = resolve_unit<IDX>(p, b);
   if (threadIdx.x == 0) raise_err(p.err, u.err);
   if (u.status == U_SKIP) return;
-  const int64_t out_at = ((int64_t)b * p.HV + hv) * p.V + myrow_v;
   if (u.status == U_PAD) {
-    if (writer) st_out1(p.out, out_at, 0.0f, (p.flags & F_OUT_BF16) != 0);
+    for (int i = 0; i < TPC; ++i)
+      if (writer)
+        st_out1(p.out, ((int64_t)b * p.HV + hv) * p.V + (tile0 + i) * VT + row0r + myrow * RPW, 0.0f,
+                (p.flags & F_OUT_BF16) != 0);
     return;
   }
 
   // all state loads first
   const int64_t head_bytes = (int64_t)K * p.V * ST::BYTES;
-  const char* src = reinterpret_cast<const char*>(p.pool) + (u.src * p.HV + hv) * head_bytes +
-                    (int64_t)row0 * ROWB + kofs * ST::BYTES;
-  typename SV::T raw[NR];
-#pragma unroll
-  for (int jj = 0; jj < NR; ++jj) raw[jj] = SV::load(src + jj * RPW * ROWB);
-  [[maybe_unused]] float sc_in = 1.0f;
+  typename SV::T rawx[TPC][NR];
+  [[maybe_unused]] float scx[TPC];
   const int n_scale = p.V / VT;
-  if constexpr (SDT == ST_FP8) sc_in = p.scales[(u.src * p.HV + hv) * n_scale + tile];
+#pragma unroll
+  for (int i = 0; i < TPC; ++i) {
+    const char* src = reinterpret_cast<const char*>(p.pool) + (u.src * p.HV + hv) * head_bytes +
+                      (int64_t)((tile0 + i) * VT + row0r) * ROWB + kofs * ST::BYTES;
+#pragma unroll
+    for (int jj = 0; jj < NR; ++jj) rawx[i][jj] = SV::load(src + jj * RPW * ROWB);
+    scx[i] = 1.0f;
+    if constexpr (SDT == ST_FP8) scx[i] = p.scales[(u.src * p.HV + hv) * n_scale + tile0 + i];
+  }
 
   // token prologue while the tile is in flight: warp 0 computes the
   // per-token scalars, every lane loads its own q/k/v entries
   float qv[EPL], kv[EPL];
   ld_in_vec<EPL>(p.q, ((int64_t)b * p.H + h) * K + kofs, in_bf16, qv);
   ld_in_vec<EPL>(p.k, ((int64_t)b * p.H + h) * K + kofs, in_bf16, kv);
-  const float v_mine = ld_in1(p.v, ((int64_t)b * p.HV + hv) * p.V + myrow_v, in_bf16);
+  float vx[TPC];
+#pragma unroll
+  for (int i = 0; i < TPC; ++i)
+    vx[i] = ld_in1(p.v, ((int64_t)b * p.HV + hv) * p.V + (tile0 + i) * VT + row0r + myrow * RPW, in_bf16);
   if (warp == 0) {
     constexpr int KPL = K / 32;
     float qn[KPL], kn[KPL];
@@ -210,6 +222,15 @@ step_tile1(const StepParams p) {
   __syncthreads();
   const float alpha = s_pro[0], beta = s_pro[1], iq = s_pro[2], ik = s_pro[3], qk = s_pro[4];
 
+#pragma unroll
+  for (int it = 0; it < TPC; ++it) {
+  // ---- tile tile0 + it
+  const int row0 = (tile0 + it) * VT + row0r;
+  const int myrow_v = row0 + myrow * RPW;
+  const int64_t out_at = ((int64_t)b * p.HV + hv) * p.V + myrow_v;
+  const float sc_in = scx[it];
+  const float v_mine = vx[it];
+  typename SV::T (&raw)[NR] = rawx[it];
   // partial k.S and q.S of every row (raw q, k; fp8: raw code values)
   float S[NR][EPL];
   float x[NV];
@@ -263,11 +284,11 @@ step_tile1(const StepParams p) {
 #pragma unroll
       for (int e = 0; e < EPL; ++e) m = absmax_acc(m, S[jj][e]);
     m = group_max<32>(fabsf(m));
-    if (lane == 0) s_amax[warp] = m;
+    if (lane == 0) s_amax[it][warp] = m;
     __syncthreads();
-    float amax = s_amax[0];
+    float amax = s_amax[it][0];
 #pragma unroll
-    for (int w = 1; w < NW; ++w) amax = fmaxf(amax, s_amax[w]);
+    for (int w = 1; w < NW; ++w) amax = fmaxf(amax, s_amax[it][w]);
     float sn, r;
     fp8_scale_of(amax, sn, r);
     const float2 r2 = make_float2(r, r);
@@ -298,7 +319,7 @@ step_tile1(const StepParams p) {
         for (int e = 0; e < EPL; ++e) S[jj][e] = 0.0f;
       }
     }
-    if (threadIdx.x == 0) p.scales[(u.dst * p.HV + hv) * n_scale + tile] = sn;
+    if (threadIdx.x == 0) p.scales[(u.dst * p.HV + hv) * n_scale + tile0 + it] = sn;
   } else {
 #pragma unroll
     for (int jj = 0; jj < NR; ++jj) {
@@ -324,6 +345,7 @@ step_tile1(const StepParams p) {
     }
   }
   if (writer) st_out1(p.out, out_at, o_mine, (p.flags & F_OUT_BF16) != 0);
+  }
 }
 
 }  // namespace gdn
