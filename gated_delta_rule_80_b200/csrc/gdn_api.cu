@@ -16,6 +16,7 @@
 #include "../../include/gdn.h"
 #include "gdn_seq.cuh"
 #include "gdn_pipe_i8.cuh"
+#include "gdn_stream_fp8.cuh"
 #include "gdn_chunk_tc.cuh"
 
 using namespace gdn;
@@ -82,17 +83,11 @@ int launch_status() {
   return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
 
-// Single-token GDN decode on a V_FIRST pool: one small CTA per tile.
+// Single-token GDN decode on a V_FIRST fp32 or bf16 pool: one small CTA per tile.
 template <int SDT, int K, int IDX>
 int launch_tile1(StepParams p, int B, cudaStream_t s) {
   using TS = Tile1Shape<SDT, K>;
   p.n_vtiles = p.V / TS::VT;
-  if constexpr (SDT == ST_FP8) {  // two tiles per CTA where the head has an even number
-    if (p.n_vtiles % 2 == 0) {
-      step_tile1<SDT, K, IDX, 2><<<dim3(p.n_vtiles / 2, p.HV, B), TS::NW * 32, 0, s>>>(p);
-      return launch_status();
-    }
-  }
   const dim3 grid(p.n_vtiles, p.HV, B);
   step_tile1<SDT, K, IDX><<<grid, TS::NW * 32, 0, s>>>(p);
   return launch_status();
@@ -166,6 +161,7 @@ int launch_one(StepParams p, int B, cudaStream_t s) {
   if constexpr (L == L_VFIRST && GATE == GATE_SCALAR) {
     if (p.T == 1) {
       if constexpr (SDT == ST_I8H) return launch_pipe<PipeI8Shape<K>>(step_pipe_i8<K, IDX>, p, B, s);
+      else if constexpr (SDT == ST_FP8) return launch_pipe<StreamFp8Shape<K>>(step_stream_fp8<K, IDX>, p, B, s);
       else return launch_tile1<SDT, K, IDX>(p, B, s);
     }
   }
@@ -261,9 +257,9 @@ __global__ void __launch_bounds__(K == 256 ? 256 : 128) fp8_quantize_kernel(cons
       x[i][4 * c] = f.x; x[i][4 * c + 1] = f.y; x[i][4 * c + 2] = f.z; x[i][4 * c + 3] = f.w;
     }
 #pragma unroll
-    for (int e = 0; e < 16; ++e) m = absmax_acc(m, x[i][e]);
+    for (int e = 0; e < 16; e += 2) m = absmax_acc2(m, x[i][e], x[i][e + 1]);
   }
-  m = group_max<32>(fabsf(m));
+  m = group_max<32>(m);
   if ((threadIdx.x & 31) == 0) s_amax[threadIdx.x >> 5] = m;
   __syncthreads();
   float amax = s_amax[0];

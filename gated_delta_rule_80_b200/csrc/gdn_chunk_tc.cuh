@@ -88,13 +88,6 @@ __device__ __forceinline__ uint4 pack_bf16x8(const float* x) {
   return make_uint4(w[0], w[1], w[2], w[3]);
 }
 
-__device__ __forceinline__ void cp_async16(void* dst, const void* src, bool valid) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_addr(dst)), "l"(src),
-               "r"(valid ? 16 : 0)
-               : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
 
 // The token inputs of the chunk starting at absolute position `base` into
 // input buffer `buf`: k rows and q rows into the [K ; Q] operand tile, v rows
@@ -210,7 +203,7 @@ __global__ void __launch_bounds__(ChunkTC::NT, 1) prefill_chunk_tc(const StepPar
     const int buf = c & 1;
     const int64_t base = base0 + (int64_t)c * C;
     const float ca = na, cb = nb;
-    cp_async_wait_all();
+    cp_async_wait<0>();
     __syncthreads();
     if (c + 1 < nchunks) {
       chunk_issue_loads(p, sm, buf ^ 1, base + C, pos_lo, pos_hi, u.tok0, h, hv);
@@ -581,7 +574,7 @@ __global__ void __launch_bounds__(ChunkTC::NT, 1) prefill_chunk_tc(const StepPar
     (void)mbar_wait(&bar, phase ^ 1u);
     (void)mbar_wait(&bar_gr, phase_gr ^ 1u);
   }
-  cp_async_wait_all();
+  cp_async_wait<0>();
   tc_fence_before_sync();
   __syncthreads();
   if (warp == 0) {

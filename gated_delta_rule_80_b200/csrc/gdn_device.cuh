@@ -93,19 +93,32 @@ __device__ __forceinline__ float round_bf16(float x) {
   return __bfloat162float(__float2bfloat16_rn(x));
 }
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
-  uint32_t l = __bfloat16_as_ushort(__float2bfloat16_rn(lo));
-  uint32_t h = __bfloat16_as_ushort(__float2bfloat16_rn(hi));
-  return l | (h << 16);
+  const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);  // one paired conversion
+  return *reinterpret_cast<const uint32_t*>(&v);
 }
 
-// fp8 E4M3 pair <-> float2 (low byte = .x). Hardware conversions: decode is
-// exact (through half); encode rounds to nearest even and saturates to 448.
-__device__ __forceinline__ float2 e4m3x2_to_float2(uint16_t pair) {
-  const __half2 h(__nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(pair), __NV_E4M3));
-  return __half22float2(h);
+// fp8 E4M3 codes: hardware conversions; decode is exact (through half),
+// encode rounds to nearest even and saturates to 448.
+// Four E4M3 bytes of a word (byte i = x[i]) <-> four floats, converting the
+// word's two halves in place (no masking or shifting to extract them).
+__device__ __forceinline__ void e4m3x4_to_float4(uint32_t w, float* x) {
+  uint32_t h0, h1;
+  asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %2;\n\t"
+      "cvt.rn.f16x2.e4m3x2 %0, lo;\n\tcvt.rn.f16x2.e4m3x2 %1, hi;\n\t}"
+      : "=r"(h0), "=r"(h1)
+      : "r"(w));
+  const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&h0));
+  const float2 b = __half22float2(*reinterpret_cast<const __half2*>(&h1));
+  x[0] = a.x; x[1] = a.y; x[2] = b.x; x[3] = b.y;
 }
-__device__ __forceinline__ uint16_t float2_to_e4m3x2(float x, float y) {
-  return static_cast<uint16_t>(__nv_cvt_float2_to_fp8x2(make_float2(x, y), __NV_SATFINITE, __NV_E4M3));
+__device__ __forceinline__ uint32_t float4_to_e4m3x4(float x0, float x1, float x2, float x3) {
+  uint32_t w;
+  asm("{\n\t.reg .b16 lo, hi;\n\t"
+      "cvt.rn.satfinite.e4m3x2.f32 lo, %2, %1;\n\tcvt.rn.satfinite.e4m3x2.f32 hi, %4, %3;\n\t"
+      "mov.b32 %0, {lo, hi};\n\t}"
+      : "=r"(w)
+      : "f"(x0), "f"(x1), "f"(x2), "f"(x3));
+  return w;
 }
 
 // ---------------------------------------------------------------------------
@@ -199,11 +212,7 @@ __device__ __forceinline__ void decode16(uint4 raw, float* x) {
     for (int i = 0; i < 4; ++i) i8x4_to_float(w[i], x + 4 * i);
   } else {
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      float2 a = e4m3x2_to_float2(static_cast<uint16_t>(w[i] & 0xffffu));
-      float2 b = e4m3x2_to_float2(static_cast<uint16_t>(w[i] >> 16));
-      x[4 * i] = a.x; x[4 * i + 1] = a.y; x[4 * i + 2] = b.x; x[4 * i + 3] = b.y;
-    }
+    for (int i = 0; i < 4; ++i) e4m3x4_to_float4(w[i], x + 4 * i);
   }
 }
 
@@ -223,42 +232,26 @@ __device__ __forceinline__ uint4 encode16(const float* x) {
     for (int i = 0; i < 4; ++i) w[i] = float_to_i8x4(x[4 * i], x[4 * i + 1], x[4 * i + 2], x[4 * i + 3]);
   } else {
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      uint32_t lo = float2_to_e4m3x2(x[4 * i], x[4 * i + 1]);
-      uint32_t hi = float2_to_e4m3x2(x[4 * i + 2], x[4 * i + 3]);
-      w[i] = lo | (hi << 16);
-    }
+    for (int i = 0; i < 4; ++i) w[i] = float4_to_e4m3x4(x[4 * i], x[4 * i + 1], x[4 * i + 2], x[4 * i + 3]);
   }
   return make_uint4(w[0], w[1], w[2], w[3]);
 }
 
 // 8 stored fp8 bytes <-> 8 floats (codes unscaled)
 __device__ __forceinline__ void decode8_fp8(uint2 raw, float* x) {
-  const uint32_t w[2] = {raw.x, raw.y};
-#pragma unroll
-  for (int i = 0; i < 2; ++i) {
-    float2 a = e4m3x2_to_float2(static_cast<uint16_t>(w[i] & 0xffffu));
-    float2 b = e4m3x2_to_float2(static_cast<uint16_t>(w[i] >> 16));
-    x[4 * i] = a.x; x[4 * i + 1] = a.y; x[4 * i + 2] = b.x; x[4 * i + 3] = b.y;
-  }
+  e4m3x4_to_float4(raw.x, x);
+  e4m3x4_to_float4(raw.y, x + 4);
 }
 __device__ __forceinline__ uint2 encode8_fp8(const float* x) {
-  uint32_t w[2];
-#pragma unroll
-  for (int i = 0; i < 2; ++i) {
-    uint32_t lo = float2_to_e4m3x2(x[4 * i], x[4 * i + 1]);
-    uint32_t hi = float2_to_e4m3x2(x[4 * i + 2], x[4 * i + 3]);
-    w[i] = lo | (hi << 16);
-  }
-  return make_uint2(w[0], w[1]);
+  return make_uint2(float4_to_e4m3x4(x[0], x[1], x[2], x[3]), float4_to_e4m3x4(x[4], x[5], x[6], x[7]));
 }
 
-// Running max of |x|: max.xorsign.abs gives max(|m|, |x|) (with the xor of
-// the signs, which the caller drops with one fabsf at the end), one
-// instruction per element instead of an abs and a max.
-__device__ __forceinline__ float absmax_acc(float m, float x) {
+// Running max of |x| (m >= 0): the absolute value is an operand modifier of
+// the max, and the three-input max of sm_100 takes two elements at once.
+__device__ __forceinline__ float absmax_acc(float m, float x) { return fmaxf(m, fabsf(x)); }
+__device__ __forceinline__ float absmax_acc2(float m, float x, float y) {
   float r;
-  asm("max.xorsign.abs.f32 %0, %1, %2;" : "=f"(r) : "f"(m), "f"(x));
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(m), "f"(fabsf(x)), "f"(fabsf(y)));
   return r;
 }
 

@@ -1,6 +1,7 @@
 // Pipeline primitives of the persistent decode kernels: shared-memory
 // mbarriers, bulk global->shared copies (cp.async.bulk, completion counted in
-// bytes on an mbarrier) and named barriers over a subset of the CTA.
+// bytes on an mbarrier), per-thread cp.async copies and named barriers over
+// a subset of the CTA.
 //
 // Every wait is bounded: after kWaitNs of global time it gives up and the
 // caller records an error, so a lost completion can never hang the GPU.
@@ -65,6 +66,21 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t by
                    smem_addr(dst)),
                "l"(src), "r"(bytes), "r"(smem_addr(bar))
                : "memory");
+}
+
+// cp.async of 16 bytes from global to shared memory (both addresses 16-byte
+// aligned), bypassing L1; `valid` false fills the 16 bytes with zeros. The
+// copies of a thread are grouped by commit and awaited by group: wait<N>
+// returns once at most N of the thread's groups are still in flight.
+__device__ __forceinline__ void cp_async16(void* dst, const void* src, bool valid) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_addr(dst)), "l"(src),
+               "r"(valid ? 16 : 0)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
 // Named barrier `id` (1..15) over the first `n` threads (a multiple of 32).

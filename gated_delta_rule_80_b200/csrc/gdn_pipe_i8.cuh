@@ -316,9 +316,13 @@ step_pipe_i8(const StepParams p, int64_t n_tiles) {
                                     __fmul2_rn(make_float2(fa[e], fa[e + 1]), make_float2(C[jj][e], C[jj][e + 1])));
         C[jj][e] = y.x;
         C[jj][e + 1] = y.y;
-        m[e] = absmax_acc(m[e], y.x);
-        m[e + 1] = absmax_acc(m[e + 1], y.y);
       }
+    }
+#pragma unroll
+    for (int e = 0; e < EPL; ++e) {
+#pragma unroll
+      for (int jj = 0; jj + 1 < NR; jj += 2) m[e] = absmax_acc2(m[e], C[jj][e], C[jj + 1][e]);
+      if constexpr (NR % 2 != 0) m[e] = absmax_acc(m[e], C[NR - 1][e]);
     }
     {
       float4* dp = reinterpret_cast<float4*>(&s_part[pid][kofs]);

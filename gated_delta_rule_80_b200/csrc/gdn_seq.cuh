@@ -191,9 +191,7 @@ step_seq(const StepParams p) {
       if constexpr (I8) {
         i8x4_to_float(raw[jj], S[jj]);
       } else {
-        const float2 a = e4m3x2_to_float2(static_cast<uint16_t>(raw[jj] & 0xffffu));
-        const float2 c = e4m3x2_to_float2(static_cast<uint16_t>(raw[jj] >> 16));
-        S[jj][0] = a.x; S[jj][1] = a.y; S[jj][2] = c.x; S[jj][3] = c.y;
+        e4m3x4_to_float4(raw[jj], S[jj]);
       }
     }
   }
@@ -435,8 +433,8 @@ step_seq(const StepParams p) {
 #pragma unroll
         for (int jj = 0; jj < NR; ++jj)
 #pragma unroll
-          for (int e = 0; e < EPL; ++e) m = absmax_acc(m, S[jj][e]);
-        m = group_max<32>(fabsf(m));
+          for (int e = 0; e < EPL; e += 2) m = absmax_acc2(m, S[jj][e], S[jj][e + 1]);
+        m = group_max<32>(m);
         const int buf = (tok - u.tok0) & 1;
         if (lane == 0) s_amax[buf][warp] = m;
         __syncthreads();
@@ -458,17 +456,13 @@ step_seq(const StepParams p) {
               y[e] = t2.x;
               y[e + 1] = t2.y;
             }
-            const uint32_t cw = (r == 0.0f) ? 0u
-                                            : (static_cast<uint32_t>(float2_to_e4m3x2(y[0], y[1])) |
-                                               (static_cast<uint32_t>(float2_to_e4m3x2(y[2], y[3])) << 16));
+            const uint32_t cw = (r == 0.0f) ? 0u : float4_to_e4m3x4(y[0], y[1], y[2], y[3]);
             codes[jj][w4] = cw;
             if (!last || stored_readout) {
-              const float2 a = e4m3x2_to_float2(static_cast<uint16_t>(cw & 0xffffu));
-              const float2 c = e4m3x2_to_float2(static_cast<uint16_t>(cw >> 16));
-              S[jj][4 * w4 + 0] = __fmul_rn(a.x, sn);
-              S[jj][4 * w4 + 1] = __fmul_rn(a.y, sn);
-              S[jj][4 * w4 + 2] = __fmul_rn(c.x, sn);
-              S[jj][4 * w4 + 3] = __fmul_rn(c.y, sn);
+              float d[4];
+              e4m3x4_to_float4(cw, d);
+#pragma unroll
+              for (int e = 0; e < 4; ++e) S[jj][4 * w4 + e] = __fmul_rn(d[e], sn);
             }
           }
         }

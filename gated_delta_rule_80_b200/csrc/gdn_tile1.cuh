@@ -1,6 +1,7 @@
-// Single-token GDN decode on V_FIRST pools: one short-lived CTA per
-// (sequence, value head, V-tile), kept small in registers so that many CTAs
-// per SM keep their state loads in flight.
+// Single-token GDN decode on V_FIRST fp32 and bf16 pools: one short-lived CTA
+// per (sequence, value head, V-tile), kept small in registers so that many
+// CTAs per SM keep their state loads in flight. The reduce-scatter and the
+// 16-byte state vectors below also serve the fp8 and int8 kernels.
 //
 // The state tile is VT rows of K contiguous elements (one value column of S
 // per row), a contiguous block in the pool. A CTA of NW warps issues every
@@ -26,14 +27,12 @@ namespace gdn {
 
 template <int SDT, int K>
 struct Tile1Shape {
-  // rows per tile: fp8 the [K, 64] scale tile; otherwise 16 KiB of fp32 state
-  static constexpr int VT = (SDT == ST_FP8) ? 64 : (K == 256 ? 16 : 32);
-  static constexpr int NW = (SDT == ST_FP8 && K == 256) ? 8 : 4;
+  // rows per tile: 16 KiB of fp32 state (8 KiB of bf16)
+  static constexpr int VT = (K == 256) ? 16 : 32;
+  static constexpr int NW = 4;
   // bytes one lane moves per row: a K=256 fp32 row needs 32 to fit a warp
   static constexpr int VB = (SDT == ST_F32 && K == 256) ? 32 : 16;
-  // resident CTAs per SM the register budget is sized for (fp8 holds 64
-  // decoded elements per thread)
-  static constexpr int MIN_CTAS = (SDT == ST_FP8) ? (NW == 8 ? 2 : 4) : 8;
+  static constexpr int MIN_CTAS = 8;  // resident CTAs per SM the registers are sized for
 };
 
 // Vector of VB stored bytes: load/store and decode/encode.
@@ -111,13 +110,11 @@ struct ReduceScatter {
   }
 };
 
-// TPC consecutive tiles of one (sequence, value head) per CTA: every state
-// load of all of them is issued before the first is computed, and the token
-// prologue is shared (fp8 uses 2: twice the bytes in flight per thread for
-// 16 more registers).
-template <int SDT, int K, int IDX, int TPC = 1>
-__global__ void __launch_bounds__(Tile1Shape<SDT, K>::NW * 32, (TPC == 1 ? Tile1Shape<SDT, K>::MIN_CTAS : 3))
+// fp32 and bf16 states (fp8 pools use step_stream_fp8 in gdn_stream_fp8.cuh).
+template <int SDT, int K, int IDX>
+__global__ void __launch_bounds__(Tile1Shape<SDT, K>::NW * 32, Tile1Shape<SDT, K>::MIN_CTAS)
 step_tile1(const StepParams p) {
+  static_assert(SDT == ST_F32 || SDT == ST_BF16, "plain states only");
   using ST = StateTraits<SDT>;
   using TS = Tile1Shape<SDT, K>;
   using SV = StateVec<SDT, TS::VB>;
@@ -135,7 +132,6 @@ step_tile1(const StepParams p) {
   constexpr int ROWB = K * ST::BYTES;  // bytes of one stored row
 
   __shared__ float s_pro[5];           // alpha, beta, q scale, k scale, q^.k^
-  __shared__ float s_amax[TPC][NW];
 
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
@@ -146,49 +142,38 @@ step_tile1(const StepParams p) {
   const bool holds_q = (vidx & 1) != 0;
   const int grp = lane - li;
   const bool writer = !holds_q && (li % REP) == 0;
-  const int tile0 = blockIdx.x * TPC;
+  const int tile = blockIdx.x;
   const int hv = blockIdx.y;
   const int b = blockIdx.z;            // T == 1: the token of sequence b is b
   const int h = hv / p.G;
   const int kofs = li * EPL;
   const bool in_bf16 = (p.flags & F_IN_BF16) != 0;
-  const int row0r = warp * NR * RPW + ri;   // tile row of row jj: row0r + jj * RPW
+  const int row0 = tile * VT + warp * NR * RPW + ri;   // value row of row jj: row0 + jj * RPW
+  const int myrow_v = row0 + myrow * RPW;
+  const int64_t out_at = ((int64_t)b * p.HV + hv) * p.V + myrow_v;
 
   const Unit u = resolve_unit<IDX>(p, b);
   if (threadIdx.x == 0) raise_err(p.err, u.err);
   if (u.status == U_SKIP) return;
   if (u.status == U_PAD) {
-    for (int i = 0; i < TPC; ++i)
-      if (writer)
-        st_out1(p.out, ((int64_t)b * p.HV + hv) * p.V + (tile0 + i) * VT + row0r + myrow * RPW, 0.0f,
-                (p.flags & F_OUT_BF16) != 0);
+    if (writer) st_out1(p.out, out_at, 0.0f, (p.flags & F_OUT_BF16) != 0);
     return;
   }
 
   // all state loads first
   const int64_t head_bytes = (int64_t)K * p.V * ST::BYTES;
-  typename SV::T rawx[TPC][NR];
-  [[maybe_unused]] float scx[TPC];
-  const int n_scale = p.V / VT;
+  const char* src = reinterpret_cast<const char*>(p.pool) + (u.src * p.HV + hv) * head_bytes +
+                    (int64_t)row0 * ROWB + kofs * ST::BYTES;
+  typename SV::T raw[NR];
 #pragma unroll
-  for (int i = 0; i < TPC; ++i) {
-    const char* src = reinterpret_cast<const char*>(p.pool) + (u.src * p.HV + hv) * head_bytes +
-                      (int64_t)((tile0 + i) * VT + row0r) * ROWB + kofs * ST::BYTES;
-#pragma unroll
-    for (int jj = 0; jj < NR; ++jj) rawx[i][jj] = SV::load(src + jj * RPW * ROWB);
-    scx[i] = 1.0f;
-    if constexpr (SDT == ST_FP8) scx[i] = p.scales[(u.src * p.HV + hv) * n_scale + tile0 + i];
-  }
+  for (int jj = 0; jj < NR; ++jj) raw[jj] = SV::load(src + jj * RPW * ROWB);
 
   // token prologue while the tile is in flight: warp 0 computes the
   // per-token scalars, every lane loads its own q/k/v entries
   float qv[EPL], kv[EPL];
   ld_in_vec<EPL>(p.q, ((int64_t)b * p.H + h) * K + kofs, in_bf16, qv);
   ld_in_vec<EPL>(p.k, ((int64_t)b * p.H + h) * K + kofs, in_bf16, kv);
-  float vx[TPC];
-#pragma unroll
-  for (int i = 0; i < TPC; ++i)
-    vx[i] = ld_in1(p.v, ((int64_t)b * p.HV + hv) * p.V + (tile0 + i) * VT + row0r + myrow * RPW, in_bf16);
+  const float v_mine = ld_in1(p.v, out_at, in_bf16);
   if (warp == 0) {
     constexpr int KPL = K / 32;
     float qn[KPL], kn[KPL];
@@ -222,16 +207,7 @@ step_tile1(const StepParams p) {
   __syncthreads();
   const float alpha = s_pro[0], beta = s_pro[1], iq = s_pro[2], ik = s_pro[3], qk = s_pro[4];
 
-#pragma unroll
-  for (int it = 0; it < TPC; ++it) {
-  // ---- tile tile0 + it
-  const int row0 = (tile0 + it) * VT + row0r;
-  const int myrow_v = row0 + myrow * RPW;
-  const int64_t out_at = ((int64_t)b * p.HV + hv) * p.V + myrow_v;
-  const float sc_in = scx[it];
-  const float v_mine = vx[it];
-  typename SV::T (&raw)[NR] = rawx[it];
-  // partial k.S and q.S of every row (raw q, k; fp8: raw code values)
+  // partial k.S and q.S of every row (raw q, k)
   float S[NR][EPL];
   float x[NV];
 #pragma unroll
@@ -249,18 +225,16 @@ step_tile1(const StepParams p) {
   }
   const float mine = ReduceScatter<NV, LPR / 2>::run(x, li);
   const float other = __shfl_xor_sync(kFull, mine, REP);
-  const float dk = (holds_q ? other : mine) * (ik * sc_in);
-  const float dq = (holds_q ? mine : other) * (iq * sc_in);
+  const float dk = (holds_q ? other : mine) * ik;
+  const float dq = (holds_q ? mine : other) * iq;
   const float u_mine = beta * (v_mine - alpha * dk);
   float o_mine = fmaf(qk, u_mine, alpha * dq);
 
-  // S' = alpha S + k^ u^T (u of each row from the lane that finished it);
-  // fp8: S holds code values, so the decay factor carries the tile scale
+  // S' = alpha S + k^ u^T (u of each row from the lane that finished it)
   float kh[EPL];
 #pragma unroll
   for (int e = 0; e < EPL; ++e) kh[e] = kv[e] * ik;
-  const float f = (SDT == ST_FP8) ? __fmul_rn(alpha, sc_in) : alpha;
-  const float2 f2 = make_float2(f, f);
+  const float2 f2 = make_float2(alpha, alpha);
 #pragma unroll
   for (int jj = 0; jj < NR; ++jj) {
     const float uj = __shfl_sync(kFull, u_mine, grp + 2 * jj * REP);
@@ -276,62 +250,16 @@ step_tile1(const StepParams p) {
   // storage format and store
   char* dst = reinterpret_cast<char*>(p.pool) + (u.dst * p.HV + hv) * head_bytes + (int64_t)row0 * ROWB +
               kofs * ST::BYTES;
-  const bool stored_readout = (p.flags & F_READOUT_STORED) != 0;
-  if constexpr (SDT == ST_FP8) {
-    float m = 0.f;
 #pragma unroll
-    for (int jj = 0; jj < NR; ++jj)
+  for (int jj = 0; jj < NR; ++jj) {
+    if constexpr (SDT == ST_BF16) {
 #pragma unroll
-      for (int e = 0; e < EPL; ++e) m = absmax_acc(m, S[jj][e]);
-    m = group_max<32>(fabsf(m));
-    if (lane == 0) s_amax[it][warp] = m;
-    __syncthreads();
-    float amax = s_amax[it][0];
-#pragma unroll
-    for (int w = 1; w < NW; ++w) amax = fmaxf(amax, s_amax[it][w]);
-    float sn, r;
-    fp8_scale_of(amax, sn, r);
-    const float2 r2 = make_float2(r, r);
-    if (r != 0.0f) {
-#pragma unroll
-      for (int jj = 0; jj < NR; ++jj) {
-        float y[EPL];
-#pragma unroll
-        for (int e = 0; e < EPL; e += 2) {
-          const float2 t = __fmul2_rn(make_float2(S[jj][e], S[jj][e + 1]), r2);
-          y[e] = t.x;
-          y[e + 1] = t.y;
-        }
-        const typename SV::T c = SV::encode(y);
-        SV::store(dst + jj * RPW * ROWB, c);
-        if (stored_readout) {
-          SV::decode(c, S[jj]);
-#pragma unroll
-          for (int e = 0; e < EPL; ++e) S[jj][e] = __fmul_rn(S[jj][e], sn);
-        }
-      }
-    } else {
-      // a zero tile stores +0 codes (no -0 from negative inputs)
-#pragma unroll
-      for (int jj = 0; jj < NR; ++jj) {
-        SV::store(dst + jj * RPW * ROWB, SV::zero());
-#pragma unroll
-        for (int e = 0; e < EPL; ++e) S[jj][e] = 0.0f;
-      }
+      for (int e = 0; e < EPL; ++e) S[jj][e] = round_bf16(S[jj][e]);
     }
-    if (threadIdx.x == 0) p.scales[(u.dst * p.HV + hv) * n_scale + tile0 + it] = sn;
-  } else {
-#pragma unroll
-    for (int jj = 0; jj < NR; ++jj) {
-      if constexpr (SDT == ST_BF16) {
-#pragma unroll
-        for (int e = 0; e < EPL; ++e) S[jj][e] = round_bf16(S[jj][e]);
-      }
-      SV::store(dst + jj * RPW * ROWB, SV::encode(S[jj]));
-    }
+    SV::store(dst + jj * RPW * ROWB, SV::encode(S[jj]));
   }
-  if constexpr (SDT != ST_F32) {
-    if (stored_readout) {
+  if constexpr (SDT == ST_BF16) {
+    if (p.flags & F_READOUT_STORED) {
       // o from the stored state: q^.S' of every row through the same reduction
 #pragma unroll
       for (int jj = 0; jj < NR; ++jj) {
@@ -345,7 +273,6 @@ step_tile1(const StepParams p) {
     }
   }
   if (writer) st_out1(p.out, out_at, o_mine, (p.flags & F_OUT_BF16) != 0);
-  }
 }
 
 }  // namespace gdn

@@ -389,6 +389,39 @@ def test_fp8_large_batch_reduced():
     gdn_slots_case(w.seed, B=24, T=1, H=w.H, HV=w.HV, K=w.K, V=w.V, num_slots=64, state_dtype="fp8_e4m3")
 
 
+@pytest.mark.parametrize("K,V", [(32, 64), (64, 128), (128, 64), (256, 128)])
+@pytest.mark.parametrize("in_dtype", ["bf16", "f32"])
+def test_slots_fp8_single_token_shapes(K, V, in_dtype):
+    """Single-token fp8 decode (the streaming kernel) for every head dim and
+    both input dtypes (bf16 and f32 token rows take different copy shapes)."""
+    gdn_slots_case(28, B=5, T=1, H=1, HV=2, K=K, V=V, num_slots=7, state_dtype="fp8_e4m3", in_dtype=in_dtype)
+
+
+def test_slots_fp8_single_token_padded_int64_no_l2norm():
+    r = gdn_slots_case(29, B=6, T=1, H=2, HV=4, K=128, V=128, num_slots=7, state_dtype="fp8_e4m3",
+                       index_dtype="i64", indices=[3, -1, 99, 0, 5, -1], use_qk_l2norm=False, scale=0.3)
+    assert r["err"] == G.GDN_FLAG_SLOT_RANGE
+    assert np.all(r["out"][[1, 2, 5]] == 0)
+    assert set(s for (s, _) in r["writes"]) == {3, 0, 5}
+
+
+def test_fp8_many_tiles_per_cta_with_padding():
+    """Enough tiles that each persistent CTA streams a few dozen of them across
+    sequence boundaries, with padded and out-of-range sequences among them;
+    checked on a sample of (sequence, head) pairs."""
+    B, H, HV, K, V, num_slots = 256, 16, 32, 128, 128, 260
+    idx = np.random.default_rng(30).permutation(num_slots)[:B].astype(np.int64)
+    idx[::7] = -1
+    idx[5] = num_slots + 3
+    r = np.random.default_rng(31)
+    units = sorted({(int(b), int(h)) for b, h in zip(r.integers(0, B, 300), r.integers(0, HV, 300))})
+    units += [(b, h) for b in (0, 5, 7) for h in (0, HV - 1)]
+    res = gdn_slots_case(30, B, 1, H, HV, K, V, num_slots, state_dtype="fp8_e4m3", indices=idx,
+                         units=sorted(set(units)))
+    assert res["err"] == G.GDN_FLAG_SLOT_RANGE
+    assert np.all(res["out"][idx < 0] == 0) and np.all(res["out"][5] == 0)
+
+
 def test_fp8_large_batch_full_size_sampled():
     w = W.WORKLOADS["fp8"]
     r = np.random.default_rng(52)
