@@ -417,12 +417,15 @@ def make_run(name, rank):
 
 def source_digest(files=None):
     """First 16 hex of the sha256 over the named kernel sources (all of csrc
-    when none are named), in sorted order."""
+    when none are named), in sorted order; None when one of them is gone."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "gated_delta_rule_80_b200", "csrc")
     names = sorted(files) if files else sorted(f for f in os.listdir(csrc) if f.endswith((".cu", ".cuh")))
     for f in names:
-        h.update(open(os.path.join(csrc, f), "rb").read())
+        path = os.path.join(csrc, f)
+        if not os.path.exists(path):
+            return None
+        h.update(open(path, "rb").read())
     return h.hexdigest()[:16]
 
 

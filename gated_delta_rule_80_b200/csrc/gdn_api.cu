@@ -15,8 +15,8 @@
 
 #include "../../include/gdn.h"
 #include "gdn_seq.cuh"
-#include "gdn_pipe_i8.cuh"
 #include "gdn_stream_fp8.cuh"
+#include "gdn_stream_i8.cuh"
 #include "gdn_chunk_tc.cuh"
 
 using namespace gdn;
@@ -93,12 +93,14 @@ int launch_tile1(StepParams p, int B, cudaStream_t s) {
   return launch_status();
 }
 
-// Single-token GDN decode on a V_FIRST int8_hadamard32 pool: persistent CTAs
-// (as many as fit on the device at once) over the (sequence, value head,
-// tile) units.
-template <class PS, class Kernel>
-int launch_pipe(Kernel kernel, StepParams p, int B, cudaStream_t s) {
+// Single-token GDN decode on a V_FIRST fp8 or int8_hadamard32 pool:
+// persistent CTAs (as many as fit on the device at once) over the (sequence,
+// value head, tile) units. One instantiation per kernel, so that each
+// kernel's shared-memory attribute and occupancy are set and cached for it.
+template <class PS, auto KERNEL>
+int launch_pipe(StepParams p, int B, cudaStream_t s) {
   static int resident[64] = {0};  // CTAs per SM, per device
+  const auto kernel = KERNEL;
   int dev = 0, sms = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64 ||
       cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
@@ -160,8 +162,8 @@ int launch_one(StepParams p, int B, cudaStream_t s) {
   constexpr bool CODED = (SDT == ST_FP8 || SDT == ST_I8H);
   if constexpr (L == L_VFIRST && GATE == GATE_SCALAR) {
     if (p.T == 1) {
-      if constexpr (SDT == ST_I8H) return launch_pipe<PipeI8Shape<K>>(step_pipe_i8<K, IDX>, p, B, s);
-      else if constexpr (SDT == ST_FP8) return launch_pipe<StreamFp8Shape<K>>(step_stream_fp8<K, IDX>, p, B, s);
+      if constexpr (SDT == ST_I8H) return launch_pipe<StreamI8Shape<K>, step_stream_i8<K, IDX>>(p, B, s);
+      else if constexpr (SDT == ST_FP8) return launch_pipe<StreamFp8Shape<K>, step_stream_fp8<K, IDX>>(p, B, s);
       else return launch_tile1<SDT, K, IDX>(p, B, s);
     }
   }

@@ -277,6 +277,16 @@ __device__ __forceinline__ float ld_in1(const void* base, int64_t i, bool bf16) 
               : reinterpret_cast<const float*>(base)[i];
 }
 
+// The 32-bit word holding input element i (bf16: the aligned pair), and the
+// element read back out of it.
+__device__ __forceinline__ const void* in_word(const void* base, int64_t i, bool bf16) {
+  return bf16 ? static_cast<const void*>(reinterpret_cast<const uint32_t*>(base) + (i >> 1))
+              : static_cast<const void*>(reinterpret_cast<const float*>(base) + i);
+}
+__device__ __forceinline__ float in_from_word(uint32_t w, int64_t i, bool bf16) {
+  return bf16 ? ((i & 1) ? bf16_hi(w) : bf16_lo(w)) : __uint_as_float(w);
+}
+
 // N contiguous input elements starting at element i (i a multiple of N,
 // base 16-byte aligned), widened to fp32.
 template <int N>

@@ -1,10 +1,11 @@
-// Pipeline primitives of the persistent decode kernels: shared-memory
-// mbarriers, bulk global->shared copies (cp.async.bulk, completion counted in
-// bytes on an mbarrier), per-thread cp.async copies and named barriers over
-// a subset of the CTA.
+// Pipeline primitives: shared-memory mbarriers (the tensor-core chunk kernel
+// waits on them for MMA completion), per-thread cp.async copies global ->
+// shared with group waits, and the division-free tile cursor of the
+// persistent streaming kernels.
 //
-// Every wait is bounded: after kWaitNs of global time it gives up and the
-// caller records an error, so a lost completion can never hang the GPU.
+// Every mbarrier wait is bounded: after kWaitNs of global time it gives up
+// and the caller records an error, so a lost completion can never hang the
+// GPU. cp.async group waits complete with the copies themselves.
 #pragma once
 
 #include <stdint.h>
@@ -24,14 +25,6 @@ __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
 // Make the initialised barriers visible to the async (bulk copy) proxy.
 __device__ __forceinline__ void mbar_fence_init() {
   asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-}
-// Arrive and announce `tx` bytes that bulk copies will complete on the barrier.
-__device__ __forceinline__ void mbar_arrive_tx(uint64_t* bar, uint32_t tx) {
-  asm volatile("mbarrier.arrive.expect_tx.release.cta.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)), "r"(tx)
-               : "memory");
-}
-__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
-  asm volatile("mbarrier.arrive.release.cta.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
 }
 __device__ __forceinline__ bool mbar_try(uint64_t* bar, uint32_t parity) {
   uint32_t ok;
@@ -59,15 +52,6 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
   return true;
 }
 
-// Bulk copy of `bytes` (a multiple of 16; both addresses 16-byte aligned)
-// from global to this CTA's shared memory, completed on `bar`.
-__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
-  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-                   smem_addr(dst)),
-               "l"(src), "r"(bytes), "r"(smem_addr(bar))
-               : "memory");
-}
-
 // cp.async of 16 bytes from global to shared memory (both addresses 16-byte
 // aligned), bypassing L1; `valid` false fills the 16 bytes with zeros. The
 // copies of a thread are grouped by commit and awaited by group: wait<N>
@@ -83,44 +67,41 @@ __device__ __forceinline__ void cp_async_wait() {
   asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
-// Named barrier `id` (1..15) over the first `n` threads (a multiple of 32).
-__device__ __forceinline__ void bar_sync(int id, int n) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
-}
-// The same, returning the OR of `pred` over the participating threads.
-__device__ __forceinline__ bool bar_or(int id, int n, bool pred) {
-  uint32_t r;
-  asm volatile(
-      "{\n\t.reg .pred a, b;\n\t"
-      "setp.ne.u32 a, %1, 0;\n\t"
-      "bar.red.or.pred b, %2, %3, a;\n\t"
-      "selp.u32 %0, 1, 0, b;\n\t}"
-      : "=r"(r)
-      : "r"(static_cast<uint32_t>(pred)), "r"(id), "r"(n)
-      : "memory");
-  return r != 0;
-}
-
-// Position (b, hv, vt) of a tile in (sequence, value head, V-tile) order,
+// Position of a tile: sequence b, value head hv (key head h, hv = h G + gi),
+// V-tile vt and the tile's index within the sequence's state (hv NVT + vt),
 // advanced one tile at a time without divisions.
-struct TileCursor {
-  int b, hv, vt;
-  __device__ __forceinline__ void init(int64_t t, int HV, int NVT) {
+struct StreamCursor {
+  int b, hv, h, gi, vt, within;
+  __device__ __forceinline__ void init(int64_t t, int HV, int NVT, int G) {
     const int64_t per_b = (int64_t)HV * NVT;
     b = static_cast<int>(t / per_b);
-    const int rem = static_cast<int>(t - (int64_t)b * per_b);
-    hv = rem / NVT;
-    vt = rem - hv * NVT;
+    within = static_cast<int>(t - (int64_t)b * per_b);
+    hv = within / NVT;
+    vt = within - hv * NVT;
+    h = hv / G;
+    gi = hv - h * G;
   }
-  __device__ __forceinline__ void next(int HV, int NVT) {
-    if (++vt == NVT) {
-      vt = 0;
-      if (++hv == HV) {
-        hv = 0;
-        ++b;
-      }
+  // what the step to the next tile changed: 0 nothing but the V-tile,
+  // 1 the value head, 2 the key head, 3 the sequence
+  __device__ __forceinline__ int next(int HV, int NVT, int G) {
+    ++within;
+    if (++vt < NVT) return 0;
+    vt = 0;
+    if (++hv == HV) {
+      hv = h = gi = within = 0;
+      ++b;
+      return 3;
     }
+    if (++gi < G) return 1;
+    gi = 0;
+    ++h;
+    return 2;
   }
 };
+
+// cp.async of 4 bytes (both addresses 4-byte aligned), cached in L1.
+__device__ __forceinline__ void cp_async4(void* dst, const void* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_addr(dst)), "l"(src) : "memory");
+}
 
 }  // namespace gdn

@@ -52,52 +52,6 @@ struct StreamFp8Shape {
   static_assert(STAGE % 16 == 0, "16-byte chunks");
 };
 
-// Position of a tile: sequence b, value head hv (key head h, hv = h G + gi),
-// V-tile vt and the tile's index within the sequence's state (hv NVT + vt),
-// advanced one tile at a time without divisions.
-struct StreamCursor {
-  int b, hv, h, gi, vt, within;
-  __device__ __forceinline__ void init(int64_t t, int HV, int NVT, int G) {
-    const int64_t per_b = (int64_t)HV * NVT;
-    b = static_cast<int>(t / per_b);
-    within = static_cast<int>(t - (int64_t)b * per_b);
-    hv = within / NVT;
-    vt = within - hv * NVT;
-    h = hv / G;
-    gi = hv - h * G;
-  }
-  // what the step to the next tile changed: 0 nothing but the V-tile,
-  // 1 the value head, 2 the key head, 3 the sequence
-  __device__ __forceinline__ int next(int HV, int NVT, int G) {
-    ++within;
-    if (++vt < NVT) return 0;
-    vt = 0;
-    if (++hv == HV) {
-      hv = h = gi = within = 0;
-      ++b;
-      return 3;
-    }
-    if (++gi < G) return 1;
-    gi = 0;
-    ++h;
-    return 2;
-  }
-};
-
-// cp.async of 4 bytes (both addresses 4-byte aligned), cached in L1.
-__device__ __forceinline__ void cp_async4(void* dst, const void* src) {
-  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_addr(dst)), "l"(src) : "memory");
-}
-// The 32-bit word holding input element i (bf16: the aligned pair), and the
-// element read back out of it.
-__device__ __forceinline__ const void* in_word(const void* base, int64_t i, bool bf16) {
-  return bf16 ? static_cast<const void*>(reinterpret_cast<const uint32_t*>(base) + (i >> 1))
-              : static_cast<const void*>(reinterpret_cast<const float*>(base) + i);
-}
-__device__ __forceinline__ float in_from_word(uint32_t w, int64_t i, bool bf16) {
-  return bf16 ? ((i & 1) ? bf16_hi(w) : bf16_lo(w)) : __uint_as_float(w);
-}
-
 template <int K, int IDX>
 __global__ void __launch_bounds__(StreamFp8Shape<K>::NT, StreamFp8Shape<K>::MIN_CTAS)
 step_stream_fp8(const StepParams p, int64_t n_tiles) {

@@ -104,7 +104,7 @@ typedef enum kda_beta_mode { KDA_BETA_LOGITS = 0, KDA_BETA_PROBABILITY = 1 } kda
 #define GDN_FLAG_PAGE_RANGE 2 /* a page id outside [0, num_slots) or a CSR position outside [0, nnz) */
 #define GDN_FLAG_PAGE_TABLE 4 /* empty page list, last_page_len outside [1, page_size], or a new page with no page before it */
 #define GDN_FLAG_SEQLENS 8    /* cu_seqlens not non-decreasing within [0, total_tokens] */
-#define GDN_FLAG_TIMEOUT 16   /* a wait of a pipelined kernel gave up after 1 s; outputs of the call are incomplete */
+#define GDN_FLAG_TIMEOUT 16   /* a bounded wait of a kernel (an MMA completion) gave up after 1 s; outputs of the call are incomplete */
 
 /* The recurrent-state pool.
  *  data:      [num_slots, HV, K, V] logically, stored per `layout` in
