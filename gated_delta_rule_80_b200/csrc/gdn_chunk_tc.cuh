@@ -21,10 +21,13 @@
 // results), the fp32 operands (diag(w) U)^T, U^T and P split into three bf16
 // terms each (hi + mid + lo carries 24 bits) and S0^T into two (hi + lo, 16
 // bits: S0 only enters k S0 and q S0, where that keeps outputs within about
-// 2e-6 of the scan), so every product is exact and the accumulation is fp32. The small triangular work (A, P, the
-// forward substitution, the outputs) runs on the CUDA cores: each of the two
-// warpgroups has one thread per value column v and takes half of the
-// columns, tokens or rows of every phase.
+// 2e-6 of the scan), so every product is exact and the accumulation is fp32.
+// The splits use the paired hardware conversion (round to nearest even); the
+// Gram, which needs only the chunk's rows, is issued as soon as they have
+// landed. The small triangular work (A, P, the forward substitution, the
+// outputs) runs on the CUDA cores: each of the two warpgroups has one thread
+// per value column v and takes half of the columns, tokens or rows of every
+// phase.
 //
 // Chunks are aligned to absolute token positions (multiples of 64), so with
 // page_size a multiple of 64 every page end is a chunk end; slots of a chunk
@@ -64,30 +67,38 @@ struct ChunkTC {
   static constexpr uint32_t T_ST = 0, T_G1 = 128, T_GR = 256, T_COLS = 512;
 };
 
-// Round to bf16 (nearest, ties to even) with integer operations: the result
-// is the float whose low 16 bits are zero. Finite inputs only.
-__device__ __forceinline__ float bf16_rne(float x) {
-  const uint32_t u = __float_as_uint(x);
-  return __uint_as_float((u + 0x7FFFu + ((u >> 16) & 1u)) & 0xFFFF0000u);
+// Splits of fp32 pairs into bf16 terms with the paired hardware conversion
+// (round to nearest, ties to even), packed as the MMA operands want them
+// (the first value in the low half). Each residual is exact in binary32, so
+// x = hi + lo to 16 bits, and x = hi + mid + lo to 24.
+__device__ __forceinline__ uint32_t bf16x2_rn(float x0, float x1) {
+  const __nv_bfloat162 h = __floats2bfloat162_rn(x0, x1);
+  return *reinterpret_cast<const uint32_t*>(&h);
 }
-
-// x = hi + mid + lo, each a bf16 (as floats); x - hi and the next residual
-// are exact in binary32
-__device__ __forceinline__ void split_bf16x3(float x, float& h, float& m, float& l) {
-  h = bf16_rne(x);
-  const float r = x - h;
-  m = bf16_rne(r);
-  l = bf16_rne(r - m);
+__device__ __forceinline__ float2 bf16x2_residual(float2 x, uint32_t h) {
+  return __fadd2_rn(x, make_float2(-bf16_lo(h), -bf16_hi(h)));
 }
-
-// 8 bf16-valued floats -> 16 bytes of bf16
-__device__ __forceinline__ uint4 pack_bf16x8(const float* x) {
-  uint32_t w[4];
+__device__ __forceinline__ void split2_bf16x2(float x0, float x1, uint32_t& hi, uint32_t& lo) {
+  hi = bf16x2_rn(x0, x1);
+  const float2 r = bf16x2_residual(make_float2(x0, x1), hi);
+  lo = bf16x2_rn(r.x, r.y);
+}
+__device__ __forceinline__ void split3_bf16x2(float x0, float x1, uint32_t& hi, uint32_t& mid, uint32_t& lo) {
+  hi = bf16x2_rn(x0, x1);
+  const float2 r = bf16x2_residual(make_float2(x0, x1), hi);
+  mid = bf16x2_rn(r.x, r.y);
+  const float2 r2 = bf16x2_residual(r, mid);
+  lo = bf16x2_rn(r2.x, r2.y);
+}
+// 8 values -> three 16-byte rows of bf16 terms
+__device__ __forceinline__ void split3_bf16x8(const float* x, uint4& h, uint4& m, uint4& l) {
+  uint32_t hw[4], mw[4], lw[4];
 #pragma unroll
-  for (int i = 0; i < 4; ++i) w[i] = __byte_perm(__float_as_uint(x[2 * i]), __float_as_uint(x[2 * i + 1]), 0x7632);
-  return make_uint4(w[0], w[1], w[2], w[3]);
+  for (int i = 0; i < 4; ++i) split3_bf16x2(x[2 * i], x[2 * i + 1], hw[i], mw[i], lw[i]);
+  h = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+  m = make_uint4(mw[0], mw[1], mw[2], mw[3]);
+  l = make_uint4(lw[0], lw[1], lw[2], lw[3]);
 }
-
 
 // The token inputs of the chunk starting at absolute position `base` into
 // input buffer `buf`: k rows and q rows into the [K ; Q] operand tile, v rows
@@ -204,7 +215,21 @@ __global__ void __launch_bounds__(ChunkTC::NT, 1) prefill_chunk_tc(const StepPar
     const int64_t base = base0 + (int64_t)c * C;
     const float ca = na, cb = nb;
     cp_async_wait<0>();
+    fence_async_smem();  // this thread's copies, to the tensor core's proxy
+    tc_fence_before_sync();
     __syncthreads();
+    // Gram = [K ; Q] K^T on the tensor cores at once: it needs only this
+    // chunk's rows, so it runs under the prologue and the state split
+    if (tid == 0) {
+      tc_fence_after_sync();
+      const unsigned char* kq0 = sm + CT::KQ + buf * CT::KQ_BYTES;
+      const uint32_t id_gr = umma_idesc_bf16(128, 64);
+#pragma unroll 1
+      for (int ks = 0; ks < D / 16; ++ks)
+        umma_bf16(tmem + CT::T_GR, umma_desc_kmajor(kq0 + ks * 256, D), umma_desc_kmajor(kq0 + ks * 256, D), id_gr,
+                  ks > 0);
+      umma_commit(&bar_gr);
+    }
     if (c + 1 < nchunks) {
       chunk_issue_loads(p, sm, buf ^ 1, base + C, pos_lo, pos_hi, u.tok0, h, hv);
       load_ab(base + C);
@@ -300,15 +325,12 @@ __global__ void __launch_bounds__(ChunkTC::NT, 1) prefill_chunk_tc(const StepPar
         }
 #pragma unroll
         for (int q8 = 0; q8 < 4; ++q8) {
-          float hh[8], ll[8];
+          uint32_t hw[4], lw[4];
 #pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            hh[e] = bf16_rne(x[8 * q8 + e]);
-            ll[e] = bf16_rne(x[8 * q8 + e] - hh[e]);
-          }
+          for (int i = 0; i < 4; ++i) split2_bf16x2(x[8 * q8 + 2 * i], x[8 * q8 + 2 * i + 1], hw[i], lw[i]);
           const uint32_t off = kmajor_offset(v, 32 * kc + 8 * q8, D);
-          *reinterpret_cast<uint4*>(sm + CT::S3 + off) = pack_bf16x8(hh);
-          *reinterpret_cast<uint4*>(sm + CT::S3 + CT::S3_BYTES + off) = pack_bf16x8(ll);
+          *reinterpret_cast<uint4*>(sm + CT::S3 + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+          *reinterpret_cast<uint4*>(sm + CT::S3 + CT::S3_BYTES + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
         }
 #pragma unroll
         for (int i = 0; i < 32; ++i) x[i] *= eC;
@@ -319,14 +341,10 @@ __global__ void __launch_bounds__(ChunkTC::NT, 1) prefill_chunk_tc(const StepPar
     tc_fence_before_sync();
     __syncthreads();
 
-    // ---- G1 = S0^T [K ; Q]^T and Gram = [K ; Q] K^T on the tensor cores
+    // ---- G1 = S0^T [K ; Q]^T on the tensor cores
     if (tid == 0) {
       tc_fence_after_sync();
-      const uint32_t id_g1 = umma_idesc_bf16(128, 128), id_gr = umma_idesc_bf16(128, 64);
-#pragma unroll 1
-      for (int ks = 0; ks < D / 16; ++ks)
-        umma_bf16(tmem + CT::T_GR, umma_desc_kmajor(kq + ks * 256, D), umma_desc_kmajor(kq + ks * 256, D), id_gr, ks > 0);
-      umma_commit(&bar_gr);
+      const uint32_t id_g1 = umma_idesc_bf16(128, 128);
 #pragma unroll 1
       for (int i = 0; i < 2; ++i)
 #pragma unroll 1
@@ -335,7 +353,7 @@ __global__ void __launch_bounds__(ChunkTC::NT, 1) prefill_chunk_tc(const StepPar
                     umma_desc_kmajor(kq + ks * 256, D), id_g1, i > 0 || ks > 0);
       umma_commit(&bar);
     }
-    // the Gram first: A, P and K^T do not wait for G1
+    // the Gram (issued first): A, P and K^T do not wait for G1
     if (wait_on(&bar_gr, phase_gr)) {
       aborted = true;
       break;
@@ -366,13 +384,12 @@ __global__ void __launch_bounds__(ChunkTC::NT, 1) prefill_chunk_tc(const StepPar
           w[e] = sx < lim ? ct * d * gr[s8 + e] : 0.0f;
         }
         if (is_p) {
-          float hh[8], mm[8], ll[8];
-#pragma unroll
-          for (int e = 0; e < 8; ++e) split_bf16x3(w[e], hh[e], mm[e], ll[e]);
+          uint4 hh, mm, ll;
+          split3_bf16x8(w, hh, mm, ll);
           const uint32_t off = kmajor_offset(t, 32 * wg + s8, C);
-          *reinterpret_cast<uint4*>(sm + CT::P3 + off) = pack_bf16x8(hh);
-          *reinterpret_cast<uint4*>(sm + CT::P3 + CT::P_BYTES + off) = pack_bf16x8(mm);
-          *reinterpret_cast<uint4*>(sm + CT::P3 + 2 * CT::P_BYTES + off) = pack_bf16x8(ll);
+          *reinterpret_cast<uint4*>(sm + CT::P3 + off) = hh;
+          *reinterpret_cast<uint4*>(sm + CT::P3 + CT::P_BYTES + off) = mm;
+          *reinterpret_cast<uint4*>(sm + CT::P3 + 2 * CT::P_BYTES + off) = ll;
         } else {
           *reinterpret_cast<float4*>(arow + s8) = make_float4(w[0], w[1], w[2], w[3]);
           *reinterpret_cast<float4*>(arow + s8 + 4) = make_float4(w[4], w[5], w[6], w[7]);
@@ -476,13 +493,15 @@ __global__ void __launch_bounds__(ChunkTC::NT, 1) prefill_chunk_tc(const StepPar
 #pragma unroll 1
     for (int tt = 0; tt < 4; ++tt) {
       const int t8 = 4 * wg + tt;
-      float hh[8], mm[8], ll[8];
+      float x[8];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) split_bf16x3(Us[(8 * t8 + i) * D + v], hh[i], mm[i], ll[i]);
+      for (int i = 0; i < 8; ++i) x[i] = Us[(8 * t8 + i) * D + v];
+      uint4 hh, mm, ll;
+      split3_bf16x8(x, hh, mm, ll);
       const uint32_t off = kmajor_offset(v, 8 * t8, C);
-      *reinterpret_cast<uint4*>(sm + CT::UT3 + off) = pack_bf16x8(hh);
-      *reinterpret_cast<uint4*>(sm + CT::UT3 + CT::UT_BYTES + off) = pack_bf16x8(mm);
-      *reinterpret_cast<uint4*>(sm + CT::UT3 + 2 * CT::UT_BYTES + off) = pack_bf16x8(ll);
+      *reinterpret_cast<uint4*>(sm + CT::UT3 + off) = hh;
+      *reinterpret_cast<uint4*>(sm + CT::UT3 + CT::UT_BYTES + off) = mm;
+      *reinterpret_cast<uint4*>(sm + CT::UT3 + 2 * CT::UT_BYTES + off) = ll;
     }
     fence_async_smem();
     tc_fence_before_sync();
@@ -523,16 +542,18 @@ __global__ void __launch_bounds__(ChunkTC::NT, 1) prefill_chunk_tc(const StepPar
 #pragma unroll 1
     for (int tt = 0; tt < 4; ++tt) {
       const int t8 = 4 * wg + tt;
-      float hh[8], mm[8], ll[8];
+      float x[8];
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
         const int t = 8 * t8 + i;
-        split_bf16x3(s_wc[t] * Us[t * D + v], hh[i], mm[i], ll[i]);
+        x[i] = s_wc[t] * Us[t * D + v];
       }
+      uint4 hh, mm, ll;
+      split3_bf16x8(x, hh, mm, ll);
       const uint32_t off = kmajor_offset(v, 8 * t8, C);
-      *reinterpret_cast<uint4*>(sm + CT::UT3 + off) = pack_bf16x8(hh);
-      *reinterpret_cast<uint4*>(sm + CT::UT3 + CT::UT_BYTES + off) = pack_bf16x8(mm);
-      *reinterpret_cast<uint4*>(sm + CT::UT3 + 2 * CT::UT_BYTES + off) = pack_bf16x8(ll);
+      *reinterpret_cast<uint4*>(sm + CT::UT3 + off) = hh;
+      *reinterpret_cast<uint4*>(sm + CT::UT3 + CT::UT_BYTES + off) = mm;
+      *reinterpret_cast<uint4*>(sm + CT::UT3 + 2 * CT::UT_BYTES + off) = ll;
     }
     fence_async_smem();
     tc_fence_before_sync();
