@@ -148,22 +148,22 @@ step_tile1(const StepParams p) {
   const int h = hv / p.G;
   const int kofs = li * EPL;
   const bool in_bf16 = (p.flags & F_IN_BF16) != 0;
-  const int row0 = tile * VT + warp * NR * RPW + ri;   // value row of row jj: row0 + jj * RPW
-  const int myrow_v = row0 + myrow * RPW;
-  const int64_t out_at = ((int64_t)b * p.HV + hv) * p.V + myrow_v;
+  const int row0r = warp * NR * RPW + ri;   // tile row of row jj: row0r + jj * RPW
 
   const Unit u = resolve_unit<IDX>(p, b);
   if (threadIdx.x == 0) raise_err(p.err, u.err);
   if (u.status == U_SKIP) return;
   if (u.status == U_PAD) {
-    if (writer) st_out1(p.out, out_at, 0.0f, (p.flags & F_OUT_BF16) != 0);
+    if (writer)
+      st_out1(p.out, ((int64_t)b * p.HV + hv) * p.V + tile * VT + row0r + myrow * RPW, 0.0f,
+              (p.flags & F_OUT_BF16) != 0);
     return;
   }
 
   // all state loads first
   const int64_t head_bytes = (int64_t)K * p.V * ST::BYTES;
   const char* src = reinterpret_cast<const char*>(p.pool) + (u.src * p.HV + hv) * head_bytes +
-                    (int64_t)row0 * ROWB + kofs * ST::BYTES;
+                    (int64_t)(tile * VT + row0r) * ROWB + kofs * ST::BYTES;
   typename SV::T raw[NR];
 #pragma unroll
   for (int jj = 0; jj < NR; ++jj) raw[jj] = SV::load(src + jj * RPW * ROWB);
@@ -173,7 +173,7 @@ step_tile1(const StepParams p) {
   float qv[EPL], kv[EPL];
   ld_in_vec<EPL>(p.q, ((int64_t)b * p.H + h) * K + kofs, in_bf16, qv);
   ld_in_vec<EPL>(p.k, ((int64_t)b * p.H + h) * K + kofs, in_bf16, kv);
-  const float v_mine = ld_in1(p.v, out_at, in_bf16);
+  const float v_mine = ld_in1(p.v, ((int64_t)b * p.HV + hv) * p.V + tile * VT + row0r + myrow * RPW, in_bf16);
   if (warp == 0) {
     constexpr int KPL = K / 32;
     float qn[KPL], kn[KPL];
@@ -248,6 +248,8 @@ step_tile1(const StepParams p) {
   }
 
   // storage format and store
+  const int row0 = tile * VT + row0r;
+  const int64_t out_at = ((int64_t)b * p.HV + hv) * p.V + row0 + myrow * RPW;
   char* dst = reinterpret_cast<char*>(p.pool) + (u.dst * p.HV + hv) * head_bytes + (int64_t)row0 * ROWB +
               kofs * ST::BYTES;
 #pragma unroll
