@@ -530,12 +530,23 @@ __global__ void __launch_bounds__(ChunkTC::NT, 1) prefill_chunk_tc(const StepPar
       float pu[32], ob[32];
       tmem_ld32(t_gr + 32 * wg, pu);
       tmem_ld32(t_g1 + C + 32 * wg, ob);
+      if (out_bf16) {
+        // bf16 outputs go through the chunk's v buffer (consumed by now) and
+        // leave as 16-byte rows after the next barrier
+        __nv_bfloat16* ost = reinterpret_cast<__nv_bfloat16*>(sm + CT::VB + buf * CT::V_BYTES);
 #pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        const int t = 32 * wg + i;
-        const int64_t pos = base + t;
-        if (pos >= pos_lo && pos < pos_hi)
-          st_out1(p.out, ((u.tok0 + (pos - pos_lo)) * p.HV + hv) * D + v, fmaf(s_egq[t], ob[i], pu[i]), out_bf16);
+        for (int i = 0; i < 32; ++i) {
+          const int t = 32 * wg + i;
+          ost[t * D + v] = __float2bfloat16_rn(fmaf(s_egq[t], ob[i], pu[i]));
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const int t = 32 * wg + i;
+          const int64_t pos = base + t;
+          if (pos >= pos_lo && pos < pos_hi)
+            st_out1(p.out, ((u.tok0 + (pos - pos_lo)) * p.HV + hv) * D + v, fmaf(s_egq[t], ob[i], pu[i]), false);
+        }
       }
     }
     // ---- update operand (diag(w) U)^T, split in three bf16 terms (tokens 32 wg ..)
@@ -558,6 +569,17 @@ __global__ void __launch_bounds__(ChunkTC::NT, 1) prefill_chunk_tc(const StepPar
     fence_async_smem();
     tc_fence_before_sync();
     __syncthreads();
+    if (out_bf16) {
+      // the staged bf16 outputs: 16 bytes (8 values of one token) per copy
+      const uint4* ost = reinterpret_cast<const uint4*>(sm + CT::VB + buf * CT::V_BYTES);
+#pragma unroll
+      for (int k = 0; k < C * D / 8 / CT::NT; ++k) {
+        const int id = tid + CT::NT * k, t = id / (D / 8), piece = id % (D / 8);
+        const int64_t pos = base + t;
+        if (pos >= pos_lo && pos < pos_hi)
+          __stcs(reinterpret_cast<uint4*>(p.out) + ((u.tok0 + (pos - pos_lo)) * p.HV + hv) * (D / 8) + piece, ost[id]);
+      }
+    }
     // ---- S^T += (diag(w) U)^T K on the tensor cores (the state was decayed above)
     if (tid == 0) {
       tc_fence_after_sync();
