@@ -361,19 +361,22 @@ __global__ void __launch_bounds__(ChunkTC::NT, 1) prefill_chunk_tc(const StepPar
 
     // ---- A and P rows from the Gram: thread (wg, r) takes columns 32 wg ..
     // 32 wg + 31 of row r (k row r < 64: A in fp32; q row r - 64: P as three
-    // bf16 tiles, the B operand of the output product)
+    // bf16 tiles, the B operand of the output product). A and K^T take space
+    // of the S0 split that G1 is still reading, so they are held in
+    // registers until G1 is done; P has a region of its own.
+    const int t_row = v & (C - 1);
+    const bool is_p = v >= C;
+    float aw[32];
     {
+      const int t = t_row;
       float gr[32];
       tmem_ld32(t_gr + 32 * wg, gr);
-      const int t = v & (C - 1);
-      const bool is_p = v >= C;
       const double gt = s_g[t];
       const float coef = is_p ? s_iq[t] : s_beta[t] * s_ik[t];
       const int lim = is_p ? t + 1 : t;  // columns s < lim are kept
       // e^{g_t - g_s} = e^{g_t} e^{-g_s} while e^{-g_C} stays finite; per pair otherwise
       const bool factored = gC > -80.0;
       const float ct = coef * (factored ? s_eg[t] : 1.0f);
-      float* arow = reinterpret_cast<float*>(sm + CT::AM) + t * CT::AS + 32 * wg;
 #pragma unroll
       for (int s8 = 0; s8 < 32; s8 += 8) {
         float w[8];
@@ -391,12 +394,13 @@ __global__ void __launch_bounds__(ChunkTC::NT, 1) prefill_chunk_tc(const StepPar
           *reinterpret_cast<uint4*>(sm + CT::P3 + CT::P_BYTES + off) = mm;
           *reinterpret_cast<uint4*>(sm + CT::P3 + 2 * CT::P_BYTES + off) = ll;
         } else {
-          *reinterpret_cast<float4*>(arow + s8) = make_float4(w[0], w[1], w[2], w[3]);
-          *reinterpret_cast<float4*>(arow + s8 + 4) = make_float4(w[4], w[5], w[6], w[7]);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) aw[s8 + e] = w[e];
         }
       }
     }
     // ---- K^T for the update: thread (wg, k) gathers 32 tokens of column k
+    uint4 ktw[4];
 #pragma unroll
     for (int tt = 0; tt < 4; ++tt) {
       const int t8 = 4 * wg + tt;
@@ -407,12 +411,23 @@ __global__ void __launch_bounds__(ChunkTC::NT, 1) prefill_chunk_tc(const StepPar
         const uint32_t hi = *reinterpret_cast<const uint16_t*>(kq + kmajor_offset(8 * t8 + 2 * i + 1, v, D));
         w[i] = lo | (hi << 16);
       }
-      *reinterpret_cast<uint4*>(sm + CT::KT + kmajor_offset(v, 8 * t8, C)) = make_uint4(w[0], w[1], w[2], w[3]);
+      ktw[tt] = make_uint4(w[0], w[1], w[2], w[3]);
     }
-    if (wait_mma()) {  // G1; also orders A, P and K^T before the reads below
+    if (wait_mma()) {  // G1; also orders P before the reads below
       aborted = true;
       break;
     }
+    // A and K^T into the space of the S0 split (read by the solve after the
+    // barrier that follows the residuals, and by the update product)
+    if (!is_p) {
+      float* arow = reinterpret_cast<float*>(sm + CT::AM) + t_row * CT::AS + 32 * wg;
+#pragma unroll
+      for (int s8 = 0; s8 < 32; s8 += 4)
+        *reinterpret_cast<float4*>(arow + s8) = make_float4(aw[s8], aw[s8 + 1], aw[s8 + 2], aw[s8 + 3]);
+    }
+#pragma unroll
+    for (int tt = 0; tt < 4; ++tt)
+      *reinterpret_cast<uint4*>(sm + CT::KT + kmajor_offset(v, 8 * (4 * wg + tt), C)) = ktw[tt];
     // U lives in the chunk's [K ; Q] buffer from here on: Us[t][v]
     float* Us = reinterpret_cast<float*>(sm + CT::KQ + buf * CT::KQ_BYTES);
     // ---- residuals R_t = beta_t (v_t - e^{g_t} k^_t S0), tokens 32 wg .. 32 wg + 31
