@@ -75,4 +75,4 @@ def test_profile_traffic_lookup_never_raises():
     assert bench.source_digest(["no_such_kernel.cuh"]) is None
     for wl in W.WORKLOADS:
         t = bench.profiled_traffic(wl)
-        assert t is None or t > 0
+        assert t is None or t >= 0  # an L2-resident workload can read no DRAM at all
