@@ -475,3 +475,16 @@ def test_prefill_paged_long_runs_int64():
     r = gdn_prefill_case(72, B=3, H=2, HV=4, K=64, V=128, page_size=16, max_len=300, index_dtype="i64",
                          fresh_every=1)
     assert r["err"] == 0 and len(r["write_pages"]) >= 3
+
+
+@pytest.mark.parametrize("state_dtype", ["fp8_e4m3", "int8_hadamard32"])
+def test_paged_coded_many_tiles_per_cta(state_dtype):
+    """Paged single-token decode of the coded states at a size where each
+    persistent CTA streams several tiles across sequences (with shared prefix
+    pages and new-page sequences), checked on a sample of (sequence, head)."""
+    B, HV = 64, 32
+    r = np.random.default_rng(33)
+    units = sorted({(int(b), int(h)) for b, h in zip(r.integers(0, B, 160), r.integers(0, HV, 160))})
+    res = gdn_paged_case(33, B=B, H=16, HV=HV, K=128, V=128, page_size=64, max_len=256, n_share=8,
+                         share_pages=2, force_lens={0: 129, 1: 129}, state_dtype=state_dtype, units=units)
+    assert res["err"] == 0
