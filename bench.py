@@ -211,21 +211,30 @@ class SlotsRun:
                                 block_v=self.w.block_v, output=self.out)
 
     def e2e_setup(self):
-        pin = lambda x: x.cpu().pin_memory()
-        self.h_in = [pin(x) for x in (self.q, self.k, self.v, self.a, self.b)]
-        self.h_idx = [pin(x) for x in self.idx]
-        self.d_in = [torch.empty_like(x) for x in (self.q, self.k, self.v, self.a, self.b)]
-        self.d_idx = torch.empty_like(self.idx[0])
+        # a step's inputs (q, k, v, a, b and the slot indices) sit in one
+        # pinned host block, each at a 256-byte offset, so that one copy moves
+        # them; the device block holds the views the call receives
+        parts = [self.q, self.k, self.v, self.a, self.b, self.idx[0]]
+        offs, n = [], 0
+        for x in parts:
+            offs.append(n)
+            n += (x.numel() * x.element_size() + 255) // 256 * 256
+        self.h_blk = [torch.empty(n, dtype=torch.uint8).pin_memory() for _ in range(self.n_rot)]
+        for r, hb in enumerate(self.h_blk):
+            for o, x in zip(offs, parts[:-1] + [self.idx[r]]):
+                nb = x.numel() * x.element_size()
+                hb[o:o + nb].copy_(x.contiguous().view(-1).view(torch.uint8).cpu())
+        self.d_blk = torch.empty(n, dtype=torch.uint8, device="cuda")
+        self.d_in = [self.d_blk[o:o + x.numel() * x.element_size()].view(x.dtype).view(x.shape)
+                     for o, x in zip(offs, parts)]
         self.h_out = torch.empty(self.out.shape, dtype=self.out.dtype).pin_memory()
-        self.h2d = sum(x.numel() * x.element_size() for x in self.h_in) + self.h_idx[0].numel() * 4
+        self.h2d = sum(x.numel() * x.element_size() for x in parts)
         self.d2h = self.h_out.numel() * self.h_out.element_size()
 
     def e2e_step(self, i):
-        for d, h in zip(self.d_in, self.h_in):
-            d.copy_(h, non_blocking=True)
-        self.d_idx.copy_(self.h_idx[i % self.n_rot], non_blocking=True)
-        q, k, v, a, b = self.d_in
-        self.G.gdn_decode_slots(q, k, v, a, b, self.A_log, self.dt_bias, self.pool, self.d_idx,
+        self.d_blk.copy_(self.h_blk[i % self.n_rot], non_blocking=True)
+        q, k, v, a, b, idx = self.d_in
+        self.G.gdn_decode_slots(q, k, v, a, b, self.A_log, self.dt_bias, self.pool, idx,
                                 state_scales=self.scales, state_layout=self.w.layout, block_v=self.w.block_v,
                                 output=self.out)
         self.h_out.copy_(self.out, non_blocking=True)

@@ -111,3 +111,18 @@ def test_int8h32_full_size_sampled():
     units = sorted({(int(b), int(h)) for b, h in zip(r.integers(0, w.B, 300), r.integers(0, w.HV, 300))})
     gdn_slots_case(w.seed, w.B, w.T, w.H, w.HV, w.K, w.V, w.num_slots, state_dtype=I8,
                    in_dtype="bf16", out_dtype="bf16", units=units)
+
+
+@pytest.mark.parametrize("K,V", [(32, 64), (64, 128), (128, 64), (256, 128), (256, 64)])
+@pytest.mark.parametrize("in_dtype", ["bf16", "f32"])
+def test_int8h32_single_token_shapes(K, V, in_dtype):
+    """Single-token V_FIRST decode (the streaming kernel) for every head dim and
+    both input dtypes (their token rows take different copy shapes)."""
+    gdn_slots_case(101, B=5, T=1, H=1, HV=2, K=K, V=V, num_slots=7, state_dtype=I8, in_dtype=in_dtype)
+
+
+def test_int8h32_single_token_padded_stored_readout_k256():
+    r = gdn_slots_case(102, B=5, T=1, H=1, HV=2, K=256, V=128, num_slots=6, state_dtype=I8,
+                       indices=[3, -1, 99, 0, 5], readout="stored", index_dtype="i64")
+    assert r["err"] == G.GDN_FLAG_SLOT_RANGE
+    assert np.all(r["out"][[1, 2]] == 0)
