@@ -163,7 +163,10 @@ int launch_one(StepParams p, int B, cudaStream_t s) {
   if constexpr (L == L_VFIRST && GATE == GATE_SCALAR) {
     if (p.T == 1) {
       if constexpr (SDT == ST_I8H) return launch_pipe<StreamI8Shape<K>, step_stream_i8<K, IDX>>(p, B, s);
-      else if constexpr (SDT == ST_FP8) return launch_pipe<StreamFp8Shape<K>, step_stream_fp8<K, IDX>>(p, B, s);
+      else if constexpr (SDT == ST_FP8) {
+        if (p.V % 128 == 0) return launch_pipe<StreamFp8Shape<K, 2>, step_stream_fp8<K, IDX, 2>>(p, B, s);
+        return launch_pipe<StreamFp8Shape<K, 1>, step_stream_fp8<K, IDX, 1>>(p, B, s);
+      }
       else return launch_tile1<SDT, K, IDX>(p, B, s);
     }
   }
