@@ -264,6 +264,28 @@ class SlotsRun:
         return done / el, f"oracle gdn_decode_slots on {nb} of {w.B} sequences x {w.HV} heads, repeated " \
                           f"{done // (nb * w.T)} times in {el:.1f} s"
 
+    def cpu_baseline_all_cores(self, seconds):
+        """The oracle on every host core: worker i takes sequences i, i+n, ...
+        of the call (n workers, at most one per sequence)."""
+        w, t = self.w, self.host_tokens
+        n = host_cores(w.B)
+        idx = W.slot_indices(self.seed, w.B, w.num_slots, 0)
+        jobs = []
+        for i in range(n):
+            rows = np.arange(i, w.B, n)
+            states, scales = W.host_pool(self.seed, idx[rows].tolist(), w.HV, w.K, w.V, w.layout, w.state_dtype,
+                                         w.block_v)
+            args = tuple(t[name][rows] for name in ("q", "k", "v", "a", "b")) + \
+                (t["A_log"], t["dt_bias"], states, idx[rows])
+            kw = dict(layout=w.layout, state_dtype=w.state_dtype, state_scales=scales, block_v=w.block_v)
+            jobs.append({"fn": "gdn_decode_slots", "args": args, "kw": kw, "tokens_per_call": len(rows) * w.T})
+        v = oracle_all_cores(jobs, seconds)
+        if v is None:
+            return None
+        return {"value": v, "unit": "tokens/s", "cores": n, "kind": "oracle",
+                "sample": f"oracle gdn_decode_slots, all {w.B} sequences x {w.HV} heads split over {n} "
+                          f"single-threaded processes, {seconds:.0f} s window"}
+
 
 class PagedRun:
     """GDN paged pool, one token (the 'paged' workload). Steps rotate over 4
@@ -421,6 +443,65 @@ def make_run(name, rank):
 
 
 # ----------------------------------------------------------------------------
+# the oracle on all host cores
+# ----------------------------------------------------------------------------
+
+def host_cores(cap):
+    """Cores this process may run on: its CPU affinity, bounded by a cgroup
+    CPU quota when one is set, and by ``cap``."""
+    n = len(os.sched_getaffinity(0))
+    try:
+        quota, period = open("/sys/fs/cgroup/cpu.max").read().split()[:2]
+        if quota != "max":
+            n = min(n, max(1, int(int(quota) // int(period))))
+    except (OSError, ValueError):
+        pass
+    return max(1, min(n, cap))
+
+
+def oracle_all_cores(jobs, seconds):
+    """Runs one oracle worker per job (``oracle.timing``), each its own
+    single-threaded interpreter, over one common wall-clock window; returns
+    the summed tokens per second, or None when a worker failed."""
+    import pickle
+    import shutil
+    import tempfile
+    env = dict(os.environ, OMP_NUM_THREADS="1", OPENBLAS_NUM_THREADS="1", MKL_NUM_THREADS="1")
+    tmp = tempfile.mkdtemp(prefix="gdn_oracle_")
+    procs = []
+    try:
+        for i, job in enumerate(jobs):
+            path = os.path.join(tmp, f"job{i}.pkl")
+            with open(path, "wb") as f:
+                pickle.dump(job, f)
+            procs.append(subprocess.Popen([sys.executable, "-m", "oracle.timing", path], cwd=ROOT, env=env,
+                                          stdin=subprocess.PIPE, stdout=subprocess.PIPE, text=True))
+        for pr in procs:
+            if pr.stdout.readline().strip() != "ready":
+                return None
+        start = time.time() + 0.5
+        window = json.dumps({"start": start, "end": start + seconds}) + "\n"
+        for pr in procs:
+            pr.stdin.write(window)
+            pr.stdin.flush()
+        done, finished = 0, start
+        for pr in procs:
+            out, _ = pr.communicate(timeout=seconds + 120)
+            if pr.returncode != 0:
+                return None
+            r = json.loads(out.strip().splitlines()[-1])
+            done += int(r["done"])
+            finished = max(finished, float(r["finished"]))
+        return done / (finished - start)
+    finally:
+        for pr in procs:
+            if pr.poll() is None:
+                pr.kill()
+                pr.wait()
+        shutil.rmtree(tmp, ignore_errors=True)
+
+
+# ----------------------------------------------------------------------------
 # roofline bookkeeping
 # ----------------------------------------------------------------------------
 
@@ -539,6 +620,9 @@ def run_b200(args, world, rank, local):
     if rank == 0 and world == 1 and not args.no_cpu_baseline and hasattr(run, "cpu_baseline"):
         v, sample = run.cpu_baseline(args.cpu_seconds)
         cpu = {"value": v, "unit": "tokens/s", "cores": 1, "kind": "oracle", "sample": sample}
+    cpu_all = None
+    if cpu is not None and hasattr(run, "cpu_baseline_all_cores"):
+        cpu_all = run.cpu_baseline_all_cores(args.cpu_seconds)
 
     if rank == 0:
         line = {
@@ -555,6 +639,7 @@ def run_b200(args, world, rank, local):
             "e2e": e2e,
             "gpu_launches": K,
             "cpu_baseline": cpu,
+            "cpu_baseline_all_cores": cpu_all,
         }
         print(json.dumps(line), flush=True)
 

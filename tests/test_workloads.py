@@ -76,3 +76,19 @@ def test_profile_traffic_lookup_never_raises():
     for wl in W.WORKLOADS:
         t = bench.profiled_traffic(wl)
         assert t is None or t >= 0  # an L2-resident workload can read no DRAM at all
+
+
+def test_oracle_all_cores_workers():
+    """The all-cores CPU baseline: separate oracle interpreters over one
+    window, summed; a worker that cannot run its job reports failure."""
+    import bench
+    B, T, H, HV, K, V = 2, 1, 1, 2, 32, 32
+    t = W.gdn_tokens(5, B, T, H, HV, K, V, "f32")
+    idx = np.array([0, 1])
+    states, _ = W.host_pool(5, idx.tolist(), HV, K, V, "V_FIRST", "f32")
+    args = tuple(t[n] for n in ("q", "k", "v", "a", "b")) + (t["A_log"], t["dt_bias"], states, idx)
+    job = {"fn": "gdn_decode_slots", "args": args, "kw": {"layout": "V_FIRST"}, "tokens_per_call": B * T}
+    v = bench.oracle_all_cores([job, job], 0.3)
+    assert v is not None and v > 0
+    assert bench.oracle_all_cores([dict(job, fn="no_such_function")], 0.3) is None
+    assert 1 <= bench.host_cores(4) <= 4
