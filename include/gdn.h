@@ -44,7 +44,7 @@
  *  - The return value is a gdn_status. GDN_ERR_INVALID_ARG: a shape, dtype,
  *    enum value, pointer or struct_size is wrong (nothing is launched, like
  *    the ValueError of kda_decode). GDN_ERR_UNSUPPORTED: a known option that
- *    this build does not implement (nothing is launched). GDN_ERR_CUDA: the
+ *    this library does not implement (nothing is launched). GDN_ERR_CUDA: the
  *    launch failed (cudaGetLastError after the launch).
  *  - Index VALUES (slots, pages, offsets) are not checked on the host, as the
  *    paged page says of precomputed slots. The kernel skips a unit whose
