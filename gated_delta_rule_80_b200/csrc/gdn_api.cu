@@ -433,7 +433,7 @@ const char* gdn_status_string(int status) {
   switch (status) {
     case GDN_OK: return "GDN_OK";
     case GDN_ERR_INVALID_ARG: return "GDN_ERR_INVALID_ARG: a shape, dtype, enum, pointer or struct_size is invalid";
-    case GDN_ERR_UNSUPPORTED: return "GDN_ERR_UNSUPPORTED: option not implemented by this build";
+    case GDN_ERR_UNSUPPORTED: return "GDN_ERR_UNSUPPORTED: option not implemented by this library";
     case GDN_ERR_CUDA: return "GDN_ERR_CUDA: the CUDA launch failed";
     default: return "unknown gdn status";
   }
