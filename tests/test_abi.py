@@ -182,3 +182,11 @@ def test_binding_rejects_cpu_tensors():
     with pytest.raises(ValueError):
         G.gdn_decode_slots(x, x, x, torch.zeros(1, 1, 1), torch.zeros(1, 1, 1), torch.zeros(1), torch.zeros(1),
                            torch.zeros(1, 1, 32, 32), torch.zeros(1, dtype=torch.int32))
+
+
+def test_missing_library_fails_loudly(monkeypatch, tmp_path):
+    """Without the built library the binding raises; there is no fallback."""
+    monkeypatch.setattr(G, "_lib", None)
+    monkeypatch.setattr(G, "LIB_PATH", str(tmp_path / "libgdn_b200.so"))
+    with pytest.raises(ImportError, match="no CPU fallback"):
+        G.lib()
