@@ -92,3 +92,27 @@ def test_oracle_all_cores_workers():
     assert v is not None and v > 0
     assert bench.oracle_all_cores([dict(job, fn="no_such_function")], 0.3) is None
     assert 1 <= bench.host_cores(4) <= 4
+
+
+def test_reference_arm_json_line():
+    """bench.py --impl reference times the oracle on the host and prints one
+    JSON line; a rank other than 0 prints nothing and exits 0."""
+    import json
+    import os
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    cmd = [sys.executable, os.path.join(root, "bench.py"), "--impl", "reference", "--steps", "2", "--warmup", "1"]
+    env = dict(os.environ, RANK="0", WORLD_SIZE="1")
+    r = subprocess.run(cmd, capture_output=True, text=True, timeout=600, cwd=root, env=env)
+    assert r.returncode == 0, r.stderr
+    lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["steps"] == 2 and d["value"] > 0
+    assert d["unit"] == "tokens/s" and d["higher_is_better"] is True
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["value"] == d["value"]
+    assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["d2h_bytes_per_step"] == 0
+    r1 = subprocess.run(cmd, capture_output=True, text=True, timeout=600, cwd=root,
+                        env=dict(os.environ, RANK="1", WORLD_SIZE="2"))
+    assert r1.returncode == 0 and not r1.stdout.strip()
