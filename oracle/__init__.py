@@ -17,6 +17,13 @@ Parity status of each function:
   beta=1 overwrites; beta=0 gives the product of decays), an independent
   transition-matrix formulation, exact rational arithmetic on tiny inputs,
   sequential == repeated single steps, and the paged and slot pool rules.
+* ``step_unit`` (the storage of bf16, fp8 and int8_hadamard32 states between
+  tokens, and the ``readout`` flag): pinned by the token write events of
+  the ModelOpt decode reference (a T-token call equals T one-token calls
+  that pass the state through the pool, bit for bit, on the slot, paged and
+  KDA drivers, and differs from encoding once at the end) and by the
+  stored readout equalling q^ times the decoded stored state, while the
+  working readout equals the fp32 step of the decoded state.
 * ``formats``: pinned by the OCP E4M3 format's defined points, by library
   conversions (torch bf16 and float8_e4m3fn casts) and by grid properties.
   The int8_hadamard32 codec: its rotation by scipy's Sylvester Hadamard

@@ -171,7 +171,13 @@ def _from_kv(kv2d, layout):
 
 
 def load_state(stored2d, layout, state_dtype, scales=None, block_v=64):
-    """Decode one stored (slot, head) state to a float64 [K, V] array."""
+    """Decode one stored (slot, head) state to a C-ordered float64 [K, V]
+    array (the same memory order whatever the layout, so that the products
+    that follow sum in the same order as on a state carried between tokens)."""
+    return np.ascontiguousarray(_load_state_any_order(stored2d, layout, state_dtype, scales, block_v))
+
+
+def _load_state_any_order(stored2d, layout, state_dtype, scales, block_v):
     if state_dtype == "f32":
         kv = np.asarray(stored2d, np.float32)
         return _to_kv(kv, layout).astype(np.float64)

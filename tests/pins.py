@@ -704,4 +704,187 @@ def pin_h32_state_decode_is_codec_around_f32_step():
         assert set(w8) == set(w32)
 
 
+# ----------------------------------------------------------------------------
+# per-token write events and the readout flag
+# (modelopt ... linear_attention.decode, recurrent_decode_reference: one
+# sequence runs with explicit token write events, and an empty call performs
+# no write; ...linear_attention.config, LinearAttentionDecodeConfig.readout:
+# 'working' or 'stored')
+# ----------------------------------------------------------------------------
+
+CODED = ("bf16", "fp8_e4m3", "int8_hadamard32")
+
+
+def _encode_kv(S_kv, state_dtype, layout):
+    """A float [K, V] state put into a pool entry of ``state_dtype`` through
+    the pinned format routines: (stored 2-D array in the layout, scales)."""
+    S32 = np.asarray(S_kv, np.float32)
+    if state_dtype == "f32":
+        return O._from_kv(S32, layout), None
+    if state_dtype == "bf16":
+        return O._from_kv(formats.f32_to_bf16_bits(S32), layout), None
+    if state_dtype == "fp8_e4m3":
+        c, s = formats.quantize_state(S32, 64)
+        return O._from_kv(c, layout), s
+    c, s = formats.quantize_state_h32(S32)
+    return O._from_kv(c, layout), s
+
+
+def _decode_entry(stored, scales, state_dtype, layout):
+    """A pool entry back to a float64 [K, V] state through the pinned format
+    routines (not through the oracle's load_state)."""
+    kv = O._to_kv(np.asarray(stored), layout)
+    if state_dtype == "f32":
+        return kv.astype(np.float64)
+    if state_dtype == "bf16":
+        return formats.bf16_bits_to_f32(kv).astype(np.float64)
+    if state_dtype == "fp8_e4m3":
+        return formats.dequantize_state(kv, scales, 64).astype(np.float64)
+    return formats.dequantize_state_h32(kv, scales).astype(np.float64)
+
+
+def _coded_pool(seed, slots, HV, K, V, state_dtype, layout):
+    """Pool and scales as dicts keyed by (slot, hv); states ~ N(0, 0.1)."""
+    r = np.random.default_rng(seed)
+    pool, scales = {}, {}
+    for s in range(slots):
+        for hv in range(HV):
+            pool[s, hv], scales[s, hv] = _encode_kv(r.standard_normal((K, V)) * 0.1, state_dtype, layout)
+    return pool, scales
+
+
+def _slots_call(t, pool, scales, idx, state_dtype, layout, readout_mode, sl=slice(None)):
+    return O.gdn_decode_slots(t["q"][:, sl], t["k"][:, sl], t["v"][:, sl], t["a"][:, sl], t["b"][:, sl],
+                              t["A_log"], t["dt_bias"], pool, idx, layout=layout, state_dtype=state_dtype,
+                              state_scales=scales, readout_mode=readout_mode)
+
+
+def _apply(pool, scales, writes):
+    pool, scales = dict(pool), dict(scales)
+    for key, (st, sc) in writes.items():
+        pool[key], scales[key] = st, sc
+    return pool, scales
+
+
+def _same_entry(x, y):
+    (a, sa), (b, sb) = x, y
+    return np.array_equal(a, b) and (sa is None and sb is None or np.array_equal(sa, sb))
+
+
+def pin_token_write_events_thread_through_the_pool():
+    """A T-token call on a bf16, fp8 or int8_hadamard32 pool equals T
+    one-token calls that pass the state through the pool between tokens,
+    bit for bit (outputs and every stored byte and scale), for either
+    readout; and it differs from carrying the state at full precision
+    across the call and encoding it once at the end, so the rounding of
+    every token is what the equality checks."""
+    B, T, H, HV, K, V = 2, 4, 1, 2, 8, 64
+    idx = [2, 0]
+    for n, sd in enumerate(CODED):
+        layout = ("V_FIRST", "K_FIRST")[n % 2]
+        t = _tiny_tokens(300 + n, B, T, H, HV, K, V)
+        pool, scales = _coded_pool(310 + n, 3, HV, K, V, sd, layout)
+        for ro in ("working", "stored"):
+            outT, wT = _slots_call(t, pool, scales, idx, sd, layout, ro)
+            p, sc = pool, scales
+            for s in range(T):
+                o1, w1 = _slots_call(t, p, sc, idx, sd, layout, ro, slice(s, s + 1))
+                assert np.array_equal(o1[:, 0], outT[:, s]), (sd, ro, s)
+                p, sc = _apply(p, sc, w1)
+            assert set(wT) == {(sl, hv) for sl in idx for hv in range(HV)}
+            for key in wT:
+                assert _same_entry(wT[key], (p[key], sc[key])), (sd, ro, key)
+        # full precision across the call, encoded once: a different pool
+        f64 = {key: O._from_kv(_decode_entry(pool[key], scales[key], sd, layout), layout) for key in pool}
+        _, w64 = O.gdn_decode_slots(t["q"], t["k"], t["v"], t["a"], t["b"], t["A_log"], t["dt_bias"], f64, idx,
+                                    layout=layout)
+        differs = 0
+        for key in wT:
+            once = _encode_kv(O._to_kv(w64[key][0], layout), sd, layout)
+            differs += not _same_entry(once, wT[key])
+        assert differs > 0, sd
+
+
+def pin_stored_readout_reads_the_stored_state():
+    """readout='stored': every token's output is q^ times the state the pool
+    holds after that token (decoded by the format routines, product by
+    loops). readout='working': the output of a one-token call equals the
+    fp32-state call on the decoded pool, and the stored payload is that
+    call's new state encoded (the codec wraps the fp32 step). The two
+    readouts differ on these coded pools."""
+    B, T, H, HV, K, V = 1, 3, 1, 2, 8, 64
+    idx = [1]
+    for n, sd in enumerate(CODED):
+        layout = ("K_FIRST", "V_FIRST")[n % 2]
+        t = _tiny_tokens(320 + n, B, T, H, HV, K, V)
+        pool, scales = _coded_pool(330 + n, 2, HV, K, V, sd, layout)
+        outS, _ = _slots_call(t, pool, scales, idx, sd, layout, "stored")
+        outW, _ = _slots_call(t, pool, scales, idx, sd, layout, "working")
+        p, sc = pool, scales
+        for s in range(T):
+            o1, w1 = _slots_call(t, p, sc, idx, sd, layout, "stored", slice(s, s + 1))
+            p, sc = _apply(p, sc, w1)
+            for hv in range(HV):
+                qh = O.l2_normalize(t["q"][0, s, 0]) / math.sqrt(K)
+                S_after = _decode_entry(p[idx[0], hv], sc[idx[0], hv], sd, layout)
+                ref = _loops_matvec(qh, S_after)
+                scale = np.max(np.abs(ref))
+                assert np.max(np.abs(o1[0, 0, hv] - ref)) <= 1e-12 * scale, (sd, s, hv)
+                assert np.max(np.abs(outS[0, s, hv] - ref)) <= 1e-12 * scale, (sd, s, hv)
+            assert np.max(np.abs(outW[0] - outS[0])) > 1e-6 * np.max(np.abs(outS[0])), sd
+        # working readout: the codec around the fp32 step, one token from the initial pool
+        dec = {key: O._from_kv(_decode_entry(pool[key], scales[key], sd, layout).astype(np.float32), layout)
+               for key in pool}
+        o32, w32 = _slots_call(t, dec, None, idx, "f32", layout, "working", slice(0, 1))
+        oW, wW = _slots_call(t, pool, scales, idx, sd, layout, "working", slice(0, 1))
+        assert np.array_equal(o32, oW), sd
+        for key in w32:
+            assert _same_entry(_encode_kv(O._to_kv(w32[key][0], layout), sd, layout), wW[key]), (sd, key)
+
+
+def pin_token_write_events_paged_and_kda():
+    """The same per-token write events on the other drivers: a paged suffix
+    (every page snapshot and the final page) and a KDA varlen sequence equal
+    one-token calls threaded through the pool, bit for bit, on bf16 and fp8
+    pools."""
+    ps, H, HV, K, V = 3, 1, 2, 8, 64
+    ind = [4, 0, 2, 5, 1]
+    L, T = 14, 7
+    last = [L - ps * (len(ind) - 1)]
+    for n, sd in enumerate(("bf16", "fp8_e4m3")):
+        pool, scales = _coded_pool(340 + n, 6, HV, K, V, sd, "V_FIRST")
+        t = _tiny_tokens(350 + n, 1, T, H, HV, K, V)
+        out, writes = O.gdn_decode_paged(t["q"], t["k"], t["v"], t["a"], t["b"], t["A_log"], t["dt_bias"], pool,
+                                         ind, [0, len(ind)], last, page_size=ps, state_dtype=sd,
+                                         state_scales=scales)
+        p, sc = pool, scales
+        for s in range(T):
+            Ls = L - T + s + 1
+            npg = -(-Ls // ps)
+            o1, w1 = O.gdn_decode_paged(t["q"][:, s:s + 1], t["k"][:, s:s + 1], t["v"][:, s:s + 1],
+                                        t["a"][:, s:s + 1], t["b"][:, s:s + 1], t["A_log"], t["dt_bias"], p,
+                                        ind[:npg], [0, npg], [Ls - ps * (npg - 1)], state_dtype=sd,
+                                        state_scales=sc)
+            assert np.array_equal(o1[0, 0], out[0, s]), (sd, s)
+            p, sc = _apply(p, sc, w1)
+        assert len({pg for (pg, _) in writes}) >= 2
+        for key in writes:
+            assert _same_entry(writes[key], (p[key], sc[key])), (sd, key)
+        # KDA: one sequence of T tokens vs T one-token sequences on the same slot
+        r = np.random.default_rng(360 + n)
+        q = r.standard_normal((T, H, K)); k = r.standard_normal((T, H, K))
+        v = r.standard_normal((T, HV, V)); g = r.standard_normal((T, HV, K))
+        bl = r.standard_normal((T, HV)); al = r.uniform(0, 2.8, HV); db = r.uniform(-1, 1, (HV, K))
+        kp, ks = _coded_pool(370 + n, 2, HV, K, V, sd, "K_FIRST")
+        oT, wT = O.kda_decode_varlen(q, k, v, g, bl, al, db, [0, T], kp, [1], state_dtype=sd, state_scales=ks)
+        p, sc = kp, ks
+        for s in range(T):
+            o1, w1 = O.kda_decode_varlen(q[s:s + 1], k[s:s + 1], v[s:s + 1], g[s:s + 1], bl[s:s + 1], al, db,
+                                         [0, 1], p, [1], state_dtype=sd, state_scales=sc)
+            assert np.array_equal(o1[0], oT[s]), (sd, s)
+            p, sc = _apply(p, sc, w1)
+        for key in wT:
+            assert _same_entry(wT[key], (p[key], sc[key])), (sd, key)
+
+
 ALL_PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]

@@ -117,7 +117,29 @@ def _h32_dequant_unrotated(codes_kv, scales):
     sc = np.asarray(scales, np.float32).T
     return (codes.reshape(K, V // 32, 32).astype(np.float32) * sc[..., None]).astype(np.float32).reshape(K, V)
 
+_ORIG_STEP_UNIT = O.step_unit
+
+
+def _step_unit_stored_ignored(S0, tokens, state_dtype, readout_mode="working", block_v=64):
+    """readout='stored' silently treated as 'working'."""
+    return _ORIG_STEP_UNIT(S0, tokens, state_dtype, "working", block_v)
+
+
+def _step_unit_encode_at_end(S0, tokens, state_dtype, readout_mode="working", block_v=64):
+    """The state is carried at full precision between tokens; only what is
+    stored (and read by a stored readout) passes through the format."""
+    S = S0
+    for (q_hat, k_hat, v, alpha, beta) in tokens:
+        o, S = O.gated_delta_step(S, q_hat, k_hat, v, alpha, beta)
+        S_st, payload = O.write_event(S, state_dtype, block_v)
+        if readout_mode == "stored" and state_dtype != "f32":
+            o = O.readout(S_st, q_hat)
+        yield o, payload
+
+
 MUTATIONS = {
+    "stored_readout_ignored": (O, "step_unit", _step_unit_stored_ignored),
+    "encode_after_last_token_only": (O, "step_unit", _step_unit_encode_at_end),
     "read_transposed": (O, "delta_read", lambda S, k: S @ k),
     "residual_sign": (O, "delta_residual", lambda v, v_old, beta: beta * (v_old - np.asarray(v, float))),
     "residual_no_beta": (O, "delta_residual", lambda v, v_old, beta: np.asarray(v, float) - v_old),
