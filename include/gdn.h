@@ -134,6 +134,14 @@ typedef struct gdn_state_pool {
 } gdn_state_pool;
 
 /* GDN decode on a slot pool: B sequences, T >= 1 tokens each.
+ * Source: flashinfer.gdn_paged.gated_delta_rule_decode_paged, Parameters
+ * (q, k, v, A_log, a, dt_bias, b, scale and use_qk_l2norm, which the page
+ * defines by gated_delta_rule_decode_pretranspose), with the state addressed by slot
+ * instead of by page; the step is Circuit.LLM.Mixer, "Gated memory"
+ * (gatedDeltaStep); the per-token storage and readout of a T > 1 suffix are
+ * modelopt...linear_attention.decode (recurrent_decode_reference: token
+ * write events) and ...linear_attention.config
+ * (LinearAttentionDecodeConfig: readout, state_codec).
  *  q, k     [B, T, H, K]   in_dtype (F32 or BF16)
  *  v        [B, T, HV, V]  in_dtype
  *  a, b     [B, T, HV]     in_dtype (gate and beta pre-activations)
@@ -168,6 +176,14 @@ int gdn_decode_slots(const gdn_decode_slots_params* p, gdn_stream_t stream);
 
 /* GDN decode of the last T tokens of every sequence on a paged pool
  * (num_slots = num_pages); a page holds the state after its last token.
+ * Source: flashinfer.gdn_paged.gated_delta_rule_decode_paged (the
+ * description's copy-on-new-page rule; Parameters: state_pool
+ * [num_pages, HV, V, K], page_indices / page_indptr CSR table,
+ * last_page_len in [1, page_size] including the decoded token, slots not
+ * checked against the table; Notes: a new-page sequence owns two pages).
+ * T > 1 is this library's reading of the same rule for a short suffix
+ * (modelopt...linear_attention.config, LinearAttentionDecodeConfig, which
+ * runs the recurrence over a suffix after a per-sequence prefix).
  *  q, k [B, T, H, K]; v [B, T, HV, V]; a, b [B, T, HV]; A_log, dt_bias [HV];
  *  page_indices [nnz], page_indptr [B+1], last_page_len [B] (index_dtype):
  *    CSR page table; the decoded tokens are the last T tokens of their
@@ -214,8 +230,14 @@ typedef struct gdn_decode_paged_params {
 
 int gdn_decode_paged(const gdn_decode_paged_params* p, gdn_stream_t stream);
 
-/* Prefill (or continued prefill) on a paged pool: append a varlen run of
- * tokens to every sequence. Sequence b gets n = cu_seqlens[b+1] - cu_seqlens[b]
+/* Prefill (or continued prefill) on a paged pool.
+ * Source: flashinfer.gdn_paged.gated_delta_rule_decode_paged, Parameters
+ * (the CSR page table is the one chunk_gated_delta_rule_paged takes); the
+ * run is the scan of single steps, Circuit.LLM.Mixer, "Gated memory"
+ * (gatedDeltaPrefill), computed in 64-token chunks where the state is fp32
+ * (modelopt...linear_attention.config, LinearAttentionConfig: chunk_size 64,
+ * exact solve).
+ * Appends a varlen run of tokens to every sequence. Sequence b gets n = cu_seqlens[b+1] - cu_seqlens[b]
  * new tokens, the last n of its L = (pages - 1) * page_size + last_page_len
  * tokens (the page table already includes them). The run is the scan of
  * single steps over its tokens. The state starts at zero when the sequence
@@ -254,6 +276,9 @@ int gdn_prefill_paged(const gdn_prefill_paged_params* p, gdn_stream_t stream);
 
 /* Resolve the (read_page, write_page) rows of a paged decode once per step,
  * to be shared by every layer's gdn_decode_paged call.
+ * Source: flashinfer.gdn_paged.gated_delta_rule_decode_paged, Parameters:
+ * slots (rows computed once for a page table and reused by the layers of a
+ * step; a decode given none computes them itself).
  *  page_indices [nnz], page_indptr [B+1], last_page_len [B] (index_dtype);
  *  slots_out [B, 2] int64 (device). Rows of malformed sequences are (-1, -1)
  *  and raise a GDN_FLAG_* bit. */
@@ -263,6 +288,8 @@ int gdn_paged_decode_slots(const void* page_indices, const void* page_indptr,
                            int64_t* slots_out, int32_t* err_flags, gdn_stream_t stream);
 
 /* KDA (per-key-channel gate) over varlen sequences on a slot pool.
+ * Source: max.nn.state_space.kda_decode (description, Parameters, Raises);
+ * the step is Circuit.LLM.Mixer, "Gated memory" (kdaLiteStep).
  *  q, k        [total_tokens, Hk, K]  in_dtype
  *  v           [total_tokens, HV, V]  in_dtype
  *  raw_gate    [total_tokens, HV, K]  in_dtype (before dt_bias is added)
@@ -296,6 +323,10 @@ typedef struct kda_decode_varlen_params {
 int kda_decode_varlen(const kda_decode_varlen_params* p, gdn_stream_t stream);
 
 /* fp8 E4M3 tile codec over n_states states of [K, V] (stored per layout).
+ * Source: modelopt...linear_attention.config, LinearAttentionConfig
+ * (state.block_v: one dynamic scale per [Dk, block_v] tile) and
+ * ...linear_attention.decode (recurrent_decode: state_format fp8_e4m3,
+ * block_v=64).
  * Per [K, block_v] tile: amax = max|x|, s = amax / 448, r = 1 / s (fp32,
  * round to nearest), code = E4M3(x * r) rounded to nearest even and
  * saturated to +-448; a tile with amax == 0 (or r not finite) stores s = 0
@@ -309,8 +340,11 @@ int gdn_state_dequantize_fp8(const uint8_t* codes, const float* scales, float* d
                              int64_t n_states, int32_t K, int32_t V, int32_t block_v,
                              int32_t layout, gdn_stream_t stream);
 
-/* int8_hadamard32 codec over n_states states of [K, V] (stored per layout),
- * the pool's code format on its own (see gdn_state_pool). Everything in
+/* int8_hadamard32 codec over n_states states of [K, V] (stored per layout).
+ * Source: modelopt...linear_attention.config, LinearAttentionConfig (the
+ * decode codec int8_hadamard32 fixes scales to one key channel and 32
+ * values) and LinearAttentionDecodeConfig.state_codec.
+ * The pool's code format on its own (see gdn_state_pool). Everything in
  * binary32 with one fixed rounding order, so results are reproducible bit
  * for bit: the 32 values of a group are rotated by the fast Walsh-Hadamard
  * butterflies of span 1, 2, 4, 8, 16 ((a, b) -> (a + b, a - b)), each then
