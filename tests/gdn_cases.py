@@ -26,20 +26,18 @@ from oracle import gdn as O
 TOL = {"f32": 1e-4, "bf16": 2e-2, "fp8_e4m3": 1e-4, "int8_hadamard32": 1e-4}
 CODED = ("fp8_e4m3", "int8_hadamard32")
 BF16_OUT = 2.0 ** -8
-# fp8 state read out from the STORED (re-encoded) state: where the two fp32
-# working states straddle an E4M3 rounding boundary the two sides store
-# neighbouring codes, and o moves by |q_i| times one E4M3 step (at most
-# 2^-3 of the element's magnitude). With unit-norm q scaled by 1/sqrt(K) and
-# a handful of such codes per tile, 1e-2 of the slice's max bounds it; the
-# output is then also checked against the stored state it was read from.
+# Outer bounds for outputs that a coded state's rounding feeds back into.
+# Where the GPU's and the oracle's binary32 working states straddle a rounding
+# boundary of the format, the two store neighbouring codes. A stored readout,
+# and every later token of a multi-token run, then moves by |q^_i| times one
+# code step (up to 2^-3 of the element for E4M3; amax / 127 of the group for
+# int8_hadamard32). That is not bounded relative to the output slice, so
+# 1e-2 is an end-to-end sanity bound only, met by the cases below. The parity
+# claim for these outputs is the conditional one in test_gpu_token_chain:
+# every token as its own call, checked at 1e-4 against the oracle started
+# from the state the GPU stored (a stored readout against q^ times that
+# stored state), codes within one step of the oracle's.
 TOL_FP8_STORED = 1e-2
-# fp8 state over a run of several tokens: the state is re-encoded after every
-# token, so a code that lands on the neighbouring E4M3 value on one side
-# (an fp32 rounding difference at a rounding boundary) is carried into the
-# later tokens' outputs; the same one-step bound applies. The stored codes
-# are still held to one step and >= 99.9% identical. The int8_hadamard32
-# state has the same mechanism with a step of amax / 127 per group, far
-# below an E4M3 step at the group's top, so the same bound holds.
 TOL_FP8_RUN = 1e-2
 
 
@@ -170,7 +168,8 @@ def check_stored_readout(out_gpu, t, idx, pool_after, scales_after, units, layou
         if not 0 <= s < num_slots:
             continue
         qh, _ = O.prepare_qk(t["q"][b, -1, O.key_head_of(hv, H, HV)], t["k"][b, -1, 0], sc, use_qk_l2norm)
-        S = O.load_state(pool_after[s, hv], layout, state_dtype, scales_after[s, hv], block_v)
+        S = O.load_state(pool_after[s, hv], layout, state_dtype,
+                         None if scales_after is None else scales_after[s, hv], block_v)
         e = slice_rel_err(out_gpu[b, -1, hv], qh @ S)
         assert e <= 1e-4, f"stored readout (b={b}, hv={hv}) is not q^T of the stored state: {e:.3g}"
 
