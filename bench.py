@@ -41,13 +41,15 @@ import workloads as W  # noqa: E402
 
 METRIC = "decode tokens/s and achieved HBM GB/s (% of ~8 TB/s) at 1×B200, by config"
 L2_BYTES = 126 * 2 ** 20
+MIN_REPS, MAX_REPS = 5, 20000
+E2E_STEPS = 64
 PROFILES = os.path.join(ROOT, "profiles")
 
 
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["b200", "reference"], default="b200")
     ap.add_argument("--workload", choices=["slots", "paged", "kda", "fp8", "int8", "tiny", "prefill"],
@@ -55,6 +57,9 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--seconds", type=float, default=1.0,
+                    help="device time each timed configuration covers (repetitions of --steps steps)")
+    ap.add_argument("--headline-only", action="store_true", help="skip the by_config entries")
     return ap.parse_args()
 
 
@@ -211,9 +216,12 @@ class SlotsRun:
                                 block_v=self.w.block_v, output=self.out)
 
     def e2e_setup(self):
-        # a step's inputs (q, k, v, a, b and the slot indices) sit in one
-        # pinned host block, each at a 256-byte offset, so that one copy moves
-        # them; the device block holds the views the call receives
+        """Buffers of the end-to-end loop. A step's inputs (q, k, v, a, b and
+        the slot indices) sit in one pinned host block, each at a 256-byte
+        offset, so that one copy moves them. Two device input blocks and two
+        output buffers alternate between steps, so that the copy of step
+        i+1's inputs and the copy of step i-1's output run on their own
+        streams while step i computes."""
         parts = [self.q, self.k, self.v, self.a, self.b, self.idx[0]]
         offs, n = [], 0
         for x in parts:
@@ -224,20 +232,61 @@ class SlotsRun:
             for o, x in zip(offs, parts[:-1] + [self.idx[r]]):
                 nb = x.numel() * x.element_size()
                 hb[o:o + nb].copy_(x.contiguous().view(-1).view(torch.uint8).cpu())
-        self.d_blk = torch.empty(n, dtype=torch.uint8, device="cuda")
-        self.d_in = [self.d_blk[o:o + x.numel() * x.element_size()].view(x.dtype).view(x.shape)
-                     for o, x in zip(offs, parts)]
-        self.h_out = torch.empty(self.out.shape, dtype=self.out.dtype).pin_memory()
+        self.d_blk = [torch.empty(n, dtype=torch.uint8, device="cuda") for _ in range(2)]
+        self.d_in = [[blk[o:o + x.numel() * x.element_size()].view(x.dtype).view(x.shape)
+                      for o, x in zip(offs, parts)] for blk in self.d_blk]
+        self.d_out = [torch.empty_like(self.out) for _ in range(2)]
+        self.h_out = [torch.empty(self.out.shape, dtype=self.out.dtype).pin_memory() for _ in range(2)]
+        self.s_h2d, self.s_d2h = torch.cuda.Stream(), torch.cuda.Stream()
+        self.ev_in = [torch.cuda.Event() for _ in range(2)]     # inputs of buffer j on the device
+        self.ev_done = [torch.cuda.Event() for _ in range(2)]   # the call that used buffer j finished
+        self.ev_out = [torch.cuda.Event() for _ in range(2)]    # output j copied to the host
         self.h2d = sum(x.numel() * x.element_size() for x in parts)
-        self.d2h = self.h_out.numel() * self.h_out.element_size()
+        self.d2h = self.h_out[0].numel() * self.h_out[0].element_size()
 
-    def e2e_step(self, i):
-        self.d_blk.copy_(self.h_blk[i % self.n_rot], non_blocking=True)
-        q, k, v, a, b, idx = self.d_in
-        self.G.gdn_decode_slots(q, k, v, a, b, self.A_log, self.dt_bias, self.pool, idx,
-                                state_scales=self.scales, state_layout=self.w.layout, block_v=self.w.block_v,
-                                output=self.out)
-        self.h_out.copy_(self.out, non_blocking=True)
+    def e2e_step(self, i, comp, first=False):
+        """Step i of the end-to-end loop: host-to-device copy of its inputs,
+        the decode call through the public binding, device-to-host copy of
+        its output; the copies wait only for what they overwrite (``first``:
+        the buffer has not been used yet in this sequence of steps)."""
+        j = i % 2
+        with torch.cuda.stream(self.s_h2d):
+            if not first:
+                self.s_h2d.wait_event(self.ev_done[j])
+            self.d_blk[j].copy_(self.h_blk[i % self.n_rot], non_blocking=True)
+            self.ev_in[j].record(self.s_h2d)
+        comp.wait_event(self.ev_in[j])
+        if not first:
+            comp.wait_event(self.ev_out[j])
+        q, k, v, a, b, idx = self.d_in[j]
+        with torch.cuda.stream(comp):
+            self.G.gdn_decode_slots(q, k, v, a, b, self.A_log, self.dt_bias, self.pool, idx,
+                                    state_scales=self.scales, state_layout=self.w.layout, block_v=self.w.block_v,
+                                    output=self.d_out[j])
+            self.ev_done[j].record(comp)
+        with torch.cuda.stream(self.s_d2h):
+            self.s_d2h.wait_event(self.ev_done[j])
+            self.h_out[j].copy_(self.d_out[j], non_blocking=True)
+            self.ev_out[j].record(self.s_d2h)
+
+    def e2e_drain(self, comp):
+        """Make ``comp`` wait for every copy in flight."""
+        comp.wait_stream(self.s_h2d)
+        comp.wait_stream(self.s_d2h)
+
+    def e2e_graph(self, n):
+        """n end-to-end steps captured into one CUDA graph: the copies from
+        and to pinned host memory and the decode calls made through the
+        public binding, with the dependencies between the three streams."""
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            comp = torch.cuda.current_stream()
+            self.s_h2d.wait_stream(comp)
+            self.s_d2h.wait_stream(comp)
+            for i in range(n):
+                self.e2e_step(i, comp, first=i < 2)
+            self.e2e_drain(comp)
+        return g
 
     def describe(self):
         return describe_slots(self.w)
@@ -431,7 +480,7 @@ class PrefillRun:
                 f"H={self.H}, HV={self.HV}, K=V={self.K}, bf16 in/out, fp32 pages (one snapshot per page)")
 
 
-def make_run(name, rank):
+def make_run(name, rank, layout=None):
     w = W.WORKLOADS.get(name)
     if name in ("slots", "fp8", "int8", "tiny"):
         return SlotsRun(w, rank)
@@ -439,7 +488,7 @@ def make_run(name, rank):
         return PagedRun(w, rank)
     if name == "prefill":
         return PrefillRun(None, rank)
-    return KdaRun(w, rank)
+    return KdaRun(w, rank, layout)
 
 
 # ----------------------------------------------------------------------------
@@ -520,19 +569,21 @@ def source_digest(files=None):
 
 
 def profiled_traffic(workload):
-    """DRAM bytes per launch from the committed ncu summary of this workload,
-    or None when the kernel sources it names changed since it was taken."""
-    path = os.path.join(PROFILES, f"gdn_decode_{workload}_ncu.md")
+    """(DRAM bytes per launch, source) from the committed ncu summary of this
+    workload: a number taken by an earlier ncu capture, not in this run, and
+    (None, None) when the kernel sources it names changed since."""
+    rel = f"profiles/gdn_decode_{workload}_ncu.md"
+    path = os.path.join(ROOT, rel)
     if not os.path.exists(path):
-        return None
+        return None, None
     text = open(path).read()
     dig = re.search(r"source_digest:\s*([0-9a-f]+)", text)
     tb = re.search(r"dram_bytes_per_launch:\s*([0-9.e+]+)", text)
     fl = re.search(r"source_files:\s*([^\n]+)", text)
     files = fl.group(1).split() if fl else None
     if not dig or not tb or dig.group(1) != source_digest(files):
-        return None
-    return float(tb.group(1))
+        return None, None
+    return float(tb.group(1)), rel + " (committed ncu capture; kernel sources unchanged since, by digest)"
 
 
 def measured_peak():
@@ -546,98 +597,182 @@ def measured_peak():
 # arms
 # ----------------------------------------------------------------------------
 
-def run_b200(args, world, rank, local):
-    import gated_delta_rule_80_b200 as G
-    G.lib()
-    run = make_run(args.workload, rank)
-    # bring the clocks up and load the kernels before capture
-    t_end = time.perf_counter() + 0.5
-    i = 0
-    while time.perf_counter() < t_end:
-        for _ in range(50):
-            run.step(i)
-            i += 1
-        torch.cuda.synchronize()
-    K = args.steps
-    # The K timed steps (and the W warm-up steps) are replayed from CUDA graphs:
-    # the launches are back to back on the device, with no host in between.
+def capture(run, n):
+    """A CUDA graph of n consecutive steps (launches back to back on the device)."""
     side = torch.cuda.Stream()
     side.wait_stream(torch.cuda.current_stream())
     with torch.cuda.stream(side):
         run.step(0)
     torch.cuda.current_stream().wait_stream(side)
-    g_warm, g_timed = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g_warm):
-        for j in range(args.warmup):
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for j in range(n):
             run.step(j)
-    with torch.cuda.graph(g_timed):
-        for j in range(K):
-            run.step(j)
+    return g
+
+
+def time_steps(run, K, warmup, world, local, min_seconds):
+    """Times exactly K steps per repetition, repeated until min_seconds of
+    device time are covered (at least MIN_REPS repetitions), with NVML
+    sampling the clocks over the whole window. Returns the median
+    repetition's milliseconds (max over ranks), all repetitions, and the
+    clock summary."""
+    t_end = time.perf_counter() + 0.3          # clocks up, kernels loaded
+    i = 0
+    while time.perf_counter() < t_end:
+        for _ in range(20):
+            run.step(i)
+            i += 1
+        torch.cuda.synchronize()
+    g_warm = capture(run, max(1, warmup))
+    g_timed = capture(run, K)
     stream = torch.cuda.current_stream()
     g_warm.replay()
     torch.cuda.synchronize()
-    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    g_timed.replay()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    est = max(e0.elapsed_time(e1), 1e-3)
+    reps = int(min(MAX_REPS, max(MIN_REPS, math.ceil(min_seconds * 1e3 / est))))
+    reps = int(max_over_ranks(reps, world))   # every rank replays the same number of times
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
     with ClockSampler(local) as clk:
         barrier(world)
         torch.cuda.synchronize()
         clk.timing(True)
-        t0.record(stream)
-        g_timed.replay()
-        t1.record(stream)
+        for a, b in evs:
+            a.record(stream)
+            g_timed.replay()
+            b.record(stream)
         torch.cuda.synchronize()
         clk.timing(False)
         barrier(world)
-    local_ms = t0.elapsed_time(t1)
-    total_ms, value = aggregate(local_ms, run.tokens_per_step, K, world)
-    ms_per_step = total_ms / K
-    kern_avg_ms = local_ms / K   # one launch per step, back to back
-    peak, peak_kind = measured_peak()
-    achieved = run.bytes_per_step / (kern_avg_ms / 1e3) / 1e9
-    traffic = profiled_traffic(args.workload)
+    ms = [a.elapsed_time(b) for a, b in evs]
+    med = max_over_ranks(statistics.median(ms), world)
     del g_warm, g_timed
+    return {"median_ms": med, "reps": reps, "ms": ms, "clocks": clk.summary()}
+
+
+def roofline_of(run, key, kern_ms, peak):
+    achieved = run.bytes_per_step / (kern_ms / 1e3) / 1e9
+    traffic, src = profiled_traffic(key)
+    return {"achieved": achieved, "frac": achieved / peak, "frac_of_8TBps": achieved / 8000.0,
+            "algorithmic_bytes_per_launch": run.bytes_per_step, "traffic": traffic, "traffic_source": src}
+
+
+# the configurations reported beside the headline, each timed like it
+BY_CONFIG = [("tiny", "tiny", {}), ("paged", "paged", {}), ("kda_k_first", "kda", {"layout": "K_FIRST"}),
+             ("kda_v_first", "kda", {"layout": "V_FIRST"}), ("fp8", "fp8", {}), ("int8", "int8", {}),
+             ("prefill", "prefill", {})]
+
+
+def run_b200(args, world, rank, local):
+    import gated_delta_rule_80_b200 as G
+    G.lib()
+    K = args.steps
+    peak, peak_kind = measured_peak()
+    run = make_run(args.workload, rank)
+    desc, tps, l2 = run.describe(), run.tokens_per_step, run.l2_note
+    tm = time_steps(run, K, args.warmup, world, local, args.seconds)
+    total_ms = tm["median_ms"]
+    value = world * run.tokens_per_step * K / (total_ms / 1e3)
+    ms_per_step = total_ms / K
+    kern_avg_ms = ms_per_step     # one launch per step, back to back
+    roof = roofline_of(run, args.workload, kern_avg_ms, peak)
+    clocks = tm["clocks"]
+    if clocks.get("sm_mhz"):
+        clocks["kernel_us_x_sm_mhz"] = kern_avg_ms * 1e3 * clocks["sm_mhz"]
 
     e2e = None
     if not args.no_e2e and hasattr(run, "e2e_setup"):
         run.e2e_setup()
-        for j in range(max(3, args.warmup)):
-            run.e2e_step(j)
-        torch.cuda.synchronize()
-        Ke = max(1, min(K, 500))
+        # E2E_STEPS steps per graph (a multiple of the 2 buffers and the
+        # rotation of host blocks); the graph is replayed back to back
+        g = run.e2e_graph(E2E_STEPS)
         stream = torch.cuda.current_stream()
-        barrier(world)
+        g.replay()
+        torch.cuda.synchronize()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
-        for j in range(Ke):
-            run.e2e_step(j)
+        g.replay()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        est = max(e0.elapsed_time(e1), 1e-3)
+        reps = int(max_over_ranks(max(2, math.ceil(args.seconds * 1e3 / est)), world))
+        barrier(world)
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for _ in range(reps):
+            g.replay()
         e1.record(stream)
         torch.cuda.synchronize()
         barrier(world)
         e_ms = max_over_ranks(e0.elapsed_time(e1), world)
+        Ke = reps * E2E_STEPS
         e2e = {"value": world * run.tokens_per_step * Ke / (e_ms / 1e3), "unit": "tokens/s",
-               "h2d_bytes_per_step": run.h2d, "d2h_bytes_per_step": run.d2h, "steps": Ke}
+               "h2d_bytes_per_step": run.h2d, "d2h_bytes_per_step": run.d2h, "steps": Ke,
+               "us_per_step": e_ms * 1e3 / Ke,
+               "pipeline": f"double-buffered: H2D of step i+1 and D2H of step i-1 on their own streams under "
+                           f"step i's kernel, every copy inside the timed window; {E2E_STEPS} steps (copies and "
+                           f"calls through the public binding) captured in one CUDA graph, replayed {reps} times"}
+        del g
+    del run
+    torch.cuda.empty_cache()
+
+    by_config = {}
+    if not args.headline_only:
+        for name, wl, kw in BY_CONFIG:
+            r = make_run(wl, rank, **kw)
+            t = time_steps(r, K, args.warmup, world, local, args.seconds)
+            us = t["median_ms"] * 1e3 / K
+            entry = {"workload": r.describe(), "us_per_launch": us,
+                     "tokens_per_s": world * r.tokens_per_step * K / (t["median_ms"] / 1e3),
+                     "tokens_per_launch": r.tokens_per_step, "repetitions": t["reps"],
+                     "launches_per_repetition": K, "l2": r.l2_note,
+                     "sm_mhz": t["clocks"].get("sm_mhz"), "clock_reasons": t["clocks"].get("reasons")}
+            # the committed kda capture is of the K_FIRST pool
+            ro = roofline_of(r, "kda" if name == "kda_k_first" else name, us / 1e3, peak)
+            entry.update({"achieved_GBps": ro["achieved"], "frac": ro["frac"],
+                          "frac_of_8TBps": ro["frac_of_8TBps"],
+                          "algorithmic_bytes_per_launch": ro["algorithmic_bytes_per_launch"],
+                          "traffic": ro["traffic"], "traffic_source": ro["traffic_source"]})
+            if getattr(r, "latency_bound", False):
+                entry["bound_note"] = r.latency_bound
+            by_config[name] = entry
+            del r
+            torch.cuda.empty_cache()
 
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline and hasattr(run, "cpu_baseline"):
-        v, sample = run.cpu_baseline(args.cpu_seconds)
-        cpu = {"value": v, "unit": "tokens/s", "cores": 1, "kind": "oracle", "sample": sample}
-    cpu_all = None
-    if cpu is not None and hasattr(run, "cpu_baseline_all_cores"):
-        cpu_all = run.cpu_baseline_all_cores(args.cpu_seconds)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        base = make_run(args.workload, rank)
+        if hasattr(base, "cpu_baseline"):
+            v, sample = base.cpu_baseline(args.cpu_seconds)
+            cpu = {"value": v, "unit": "tokens/s", "cores": 1, "kind": "oracle", "sample": sample}
+        cpu_all = base.cpu_baseline_all_cores(args.cpu_seconds) if hasattr(base, "cpu_baseline_all_cores") else None
+        del base
+    else:
+        cpu_all = None
 
     if rank == 0:
         line = {
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f32", "data": "synthetic (seeded; no dataset on the pages)",
-            "config": {"workload": run.describe(), "tokens_per_step_per_gpu": run.tokens_per_step,
-                       "l2": run.l2_note, "parallelism": f"independent sequences per GPU x{world}"},
-            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                         "frac": achieved / peak, "traffic": traffic, "peak_kind": peak_kind,
-                         "algorithmic_bytes_per_launch": run.bytes_per_step,
-                         "kernel_avg_us": kern_avg_ms * 1e3, "frac_of_8TBps": achieved / 8000.0},
-            "clocks": clk.summary(),
+            "config": {"workload": desc, "tokens_per_step_per_gpu": tps,
+                       "l2": l2, "parallelism": f"independent sequences per GPU x{world}",
+                       "timing": f"median of {tm['reps']} repetitions of {K} graph-replayed steps "
+                                 f"(>= {args.seconds:g} s of device time)"},
+            "roofline": {"bound": "hbm", "achieved": roof["achieved"], "peak": peak, "unit": "GB/s",
+                         "frac": roof["frac"], "traffic": roof["traffic"], "traffic_source": roof["traffic_source"],
+                         "peak_kind": peak_kind,
+                         "algorithmic_bytes_per_launch": roof["algorithmic_bytes_per_launch"],
+                         "kernel_avg_us": kern_avg_ms * 1e3, "frac_of_8TBps": roof["frac_of_8TBps"]},
+            "clocks": clocks,
             "e2e": e2e,
-            "gpu_launches": K,
+            "gpu_launches": K * tm["reps"],
+            "by_config": by_config,
             "cpu_baseline": cpu,
             "cpu_baseline_all_cores": cpu_all,
         }

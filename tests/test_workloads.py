@@ -74,8 +74,10 @@ def test_profile_traffic_lookup_never_raises():
     import bench
     assert bench.source_digest(["no_such_kernel.cuh"]) is None
     for wl in W.WORKLOADS:
-        t = bench.profiled_traffic(wl)
+        t, src = bench.profiled_traffic(wl)
         assert t is None or t >= 0  # an L2-resident workload can read no DRAM at all
+        assert (src is None) == (t is None)
+        assert src is None or src.startswith(f"profiles/gdn_decode_{wl}_ncu.md")
 
 
 def test_oracle_all_cores_workers():
