@@ -8,7 +8,7 @@ back in place. Steps rotate over 4 disjoint sets of 64 slots (512 MiB of
 state per cycle, 4x the L2), so no step finds its state in L2.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl b200|reference]
-                    [--workload slots|paged|kda|fp8|int8|tiny|prefill]
+                    [--workload slots|paged|kda|kda_long|fp8|int8|tiny|prefill]
 
 Prints one JSON line (rank 0). Under torchrun each rank runs its own batch
 on its own GPU (weak scaling; the sequences are independent, no data-path
@@ -52,7 +52,7 @@ def parse():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["b200", "reference"], default="b200")
-    ap.add_argument("--workload", choices=["slots", "paged", "kda", "fp8", "int8", "tiny", "prefill"],
+    ap.add_argument("--workload", choices=["slots", "paged", "kda", "kda_long", "fp8", "int8", "tiny", "prefill"],
                     default="slots")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
@@ -407,7 +407,7 @@ class KdaRun:
         self.G, self.w = G, w
         seed = w.seed + 1000 * rank
         self.layout = layout or w.layout
-        self.cu = W.varlen_offsets(seed, w.B, w.max_len)
+        self.cu = W.varlen_offsets(seed, w.B, w.max_len, w.min_len)
         total = int(self.cu[-1])
         t = W.kda_tokens(seed, total, w.H, w.HV, w.K, w.V, w.in_dtype)
         self.ins = [in_t(t[n], w.in_dtype) for n in ("q", "k", "v", "raw_gate", "beta_logits")]
@@ -431,7 +431,7 @@ class KdaRun:
 
     def describe(self):
         w = self.w
-        return (f"KDA varlen decode: {w.B} sequences x U[1,{w.max_len}] tokens ({self.tokens_per_step} tokens), "
+        return (f"KDA varlen decode: {w.B} sequences x U[{w.min_len},{w.max_len}] tokens ({self.tokens_per_step} tokens), "
                 f"Hk=HV={w.HV}, K=V={w.K}, bf16 inputs, fp32 state_pool [{w.num_slots},{w.HV},{w.K},{w.V}] "
                 f"{self.layout}")
 
@@ -664,8 +664,8 @@ def roofline_of(run, key, kern_ms, peak):
 
 # the configurations reported beside the headline, each timed like it
 BY_CONFIG = [("tiny", "tiny", {}), ("paged", "paged", {}), ("kda_k_first", "kda", {"layout": "K_FIRST"}),
-             ("kda_v_first", "kda", {"layout": "V_FIRST"}), ("fp8", "fp8", {}), ("int8", "int8", {}),
-             ("prefill", "prefill", {})]
+             ("kda_v_first", "kda", {"layout": "V_FIRST"}), ("kda_long", "kda_long", {}), ("fp8", "fp8", {}),
+             ("int8", "int8", {}), ("prefill", "prefill", {})]
 
 
 def run_b200(args, world, rank, local):

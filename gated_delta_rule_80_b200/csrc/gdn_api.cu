@@ -18,6 +18,7 @@
 #include "gdn_stream_fp8.cuh"
 #include "gdn_stream_i8.cuh"
 #include "gdn_chunk_tc.cuh"
+#include "gdn_kda_chunk.cuh"
 
 using namespace gdn;
 
@@ -143,6 +144,38 @@ int launch_prefill_tc(StepParams p, int B, cudaStream_t s) {
   p.G = p.HV / p.H;
   prefill_chunk_tc<<<dim3(p.HV, B), ChunkTC::NT, ChunkTC::SMEM, s>>>(p);
   return launch_status();
+}
+
+// KDA varlen on the tensor cores (fp32 pools of either layout, K = V = 128,
+// bf16 token inputs): one CTA per (value head, sequence), 32-token chunks.
+// Runs shorter than a chunk are padded, so kda_decode_varlen sends a call
+// here only when its runs average at least kKdaChunkMinMean tokens.
+constexpr int kKdaChunkMinMean = 32;
+
+template <int L>
+int launch_kda_tc_l(StepParams p, int B, cudaStream_t s) {
+  static bool ready[64] = {false};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+    cudaGetLastError();
+    return GDN_ERR_CUDA;
+  }
+  if (!ready[dev]) {
+    if (cudaFuncSetAttribute(kda_chunk_tc<L>, cudaFuncAttributeMaxDynamicSharedMemorySize, KdaTC::SMEM) !=
+        cudaSuccess) {
+      cudaGetLastError();
+      return GDN_ERR_CUDA;
+    }
+    ready[dev] = true;
+  }
+  if (B > 65535) return GDN_ERR_INVALID_ARG;  // grid y
+  p.G = p.HV / p.H;
+  kda_chunk_tc<L><<<dim3(p.HV, B), KdaTC::NT, KdaTC::SMEM, s>>>(p);
+  return launch_status();
+}
+
+int launch_kda_tc(const StepParams& p, int layout, int B, cudaStream_t s) {
+  return layout == GDN_V_FIRST ? launch_kda_tc_l<L_VFIRST>(p, B, s) : launch_kda_tc_l<L_KFIRST>(p, B, s);
 }
 
 // T >= 1 tokens per unit, either layout: the chunked-prologue kernel.
@@ -598,7 +631,11 @@ int kda_decode_varlen(const kda_decode_varlen_params* p, gdn_stream_t stream) {
   k.flags = (p->in_dtype == GDN_BF16 ? F_IN_BF16 : 0) | (p->out_dtype == GDN_BF16 ? F_OUT_BF16 : 0) | F_L2NORM |
             F_VARLEN | (p->beta_mode == KDA_BETA_PROBABILITY ? F_BETA_PROB : 0) |
             (p->readout == GDN_READOUT_STORED ? F_READOUT_STORED : 0);
-  return launch_step<GATE_VECTOR, IDX_SLOTS>(k, p->pool, p->K, p->B, reinterpret_cast<cudaStream_t>(stream));
+  const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (p->pool.dtype == GDN_F32 && p->K == 128 && p->V == 128 && p->in_dtype == GDN_BF16 &&
+      static_cast<int64_t>(p->total_tokens) >= static_cast<int64_t>(kKdaChunkMinMean) * p->B)
+    return launch_kda_tc(k, p->pool.layout, p->B, s);
+  return launch_step<GATE_VECTOR, IDX_SLOTS>(k, p->pool, p->K, p->B, s);
 }
 
 int gdn_state_quantize_fp8(const float* src, uint8_t* codes, float* scales, int64_t n_states, int32_t K, int32_t V,

@@ -19,6 +19,9 @@ Workloads (sizes and distributions of the decode problems the pages pose):
 * ``kda``   KDA varlen, 32 sequences of U[1, 8] tokens, Hk=HV=32,
   K=V=128, bf16 q/k/v/raw_gate/beta_logits, fp32 pool [64, 32, 128, 128];
   K_FIRST then V_FIRST; seed 3.
+* ``kda_long`` KDA varlen with long runs (a prefill): 8 sequences of
+  U[512, 1024] tokens, otherwise as ``kda``, fp32 pool [8, 32, 128, 128]
+  K_FIRST; seed 6.
 * ``fp8``   GDN slot pool, T=1, B=1024, H=16, HV=32, K=V=128, bf16 inputs,
   fp8_e4m3 pool [1024, 32, 128, 128] with one fp32 scale per [128, 64] tile,
   indices a random permutation of 1024; seed 4.
@@ -59,7 +62,8 @@ class Workload:
     layout: str               # 'K_FIRST' | 'V_FIRST'
     num_slots: int = 0        # slot pools
     page_size: int = 0        # paged pools
-    max_len: int = 0          # paged: lengths U[2, max_len]; kda: tokens U[1, max_len]
+    max_len: int = 0          # paged: lengths U[2, max_len]; kda: tokens U[min_len, max_len]
+    min_len: int = 1          # kda: shortest run
     n_share: int = 0          # paged: sequences sharing the prefix
     share_pages: int = 0      # paged: full pages in the shared prefix
     block_v: int = 64
@@ -76,6 +80,9 @@ WORKLOADS: Dict[str, Workload] = {
     "kda": Workload("kda", "kda_varlen", 3, B=32, T=0, H=32, HV=32, K=128, V=128,
                     in_dtype="bf16", state_dtype="f32", layout="K_FIRST", num_slots=64,
                     max_len=8),
+    "kda_long": Workload("kda_long", "kda_varlen", 6, B=8, T=0, H=32, HV=32, K=128, V=128,
+                         in_dtype="bf16", state_dtype="f32", layout="K_FIRST", num_slots=8,
+                         max_len=1024, min_len=512),
     "fp8": Workload("fp8", "gdn_slots", 4, B=1024, T=1, H=16, HV=32, K=128, V=128,
                     in_dtype="bf16", state_dtype="fp8_e4m3", layout="V_FIRST",
                     num_slots=1024, block_v=64),
