@@ -24,9 +24,8 @@
 // The operands are split into bf16 terms so that the products keep fp32
 // accuracy: S0^T and the scaled rows K~, Q~, K^ in two terms (16 bits), U
 // and P in three (24 bits); a numpy model of this kernel stays within 1e-5
-// of the float64 scan over 200 tokens. A and P (one exponential per pair
-// and key channel, exact per channel) and the solve run on the CUDA cores,
-// A and P while G1 runs.
+// of the float64 scan over 200 tokens. A and P (exact per channel) and the
+// solve run on the CUDA cores, A and P while G1 runs.
 //
 // Runs are cut into chunks from their first token; the slots of the last
 // chunk past the run are padding (k = q = v = 0, alpha = 1, beta = 0),
@@ -54,10 +53,11 @@ struct KdaTC {
   static constexpr uint32_t GM = RAW + 2 * RAW_BYTES;   // [C x GS] fp32: G in log2 units
   static constexpr uint32_t KQT = GM + C * GS * 4;      // 2 terms x [64 x 128] bf16, K-major: [K~ ; Q~]
   static constexpr uint32_t KQT_BYTES = 2 * C * D * 2;
-  static constexpr uint32_t KBT = KQT + 2 * KQT_BYTES;  // 2 buffers x 2 terms x [128 x 32] bf16, K-major: K^ ^T
+  static constexpr uint32_t KBT = KQT + 2 * KQT_BYTES;  // 2 terms x [128 x 32] bf16, K-major: K^ ^T
   static constexpr uint32_t KBT_BYTES = D * C * 2;
+  static constexpr uint32_t AL = KBT + 2 * KBT_BYTES;   // [C x GS] fp32: alpha_t[i] = 2^(G_t - G_(t-1))
   static constexpr int AS = C + 4;                      // row stride (floats) of A
-  static constexpr uint32_t AM = KBT + 4 * KBT_BYTES;   // [C x AS] fp32
+  static constexpr uint32_t AM = AL + C * GS * 4;       // [C x AS] fp32
   static constexpr uint32_t P3 = AM + C * AS * 4;       // 3 terms x [32 x 32] bf16, K-major: P
   static constexpr uint32_t P_BYTES = C * C * 2;
   // the S0^T split (2 terms x [128 x 128] bf16, K-major); once G1 is done
@@ -69,7 +69,8 @@ struct KdaTC {
   static constexpr uint32_t UT_BYTES = D * C * 2;
   static constexpr uint32_t SMEM = X + 2 * S_BYTES;
   static_assert(UT3 + 3 * UT_BYTES <= SMEM, "U and its split fit where the S0 split was");
-  static_assert(KQT % 16 == 0 && KBT % 16 == 0 && P3 % 16 == 0 && X % 16 == 0 && UT3 % 16 == 0, "16-byte tiles");
+  static_assert(KQT % 16 == 0 && KBT % 16 == 0 && AL % 16 == 0 && P3 % 16 == 0 && X % 16 == 0 && UT3 % 16 == 0,
+                "16-byte tiles");
   // tensor memory columns: state, G1 (32 k columns then 32 q columns), O
   static constexpr uint32_t T_ST = 0, T_G1 = 128, T_O = 192, T_COLS = 256;
 };
@@ -82,6 +83,21 @@ __device__ __forceinline__ float ex2_approx(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// log2(x) on the special-function unit (relative error about 2^-22).
+__device__ __forceinline__ float lg2_approx(float x) {
+  float y;
+  asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// softplus(x) / ln 2 = max(x, 0) log2(e) + log2(1 + 2^(-|x| log2(e))): the
+// decay exponent in log2 units. When 1 + 2^(...) rounds to 1 (x < -17) the
+// term it drops is below 6e-8, which moves a decay factor by less than
+// 1e-6 relative.
+__device__ __forceinline__ float softplus_log2(float x) {
+  return fmaxf(x, 0.0f) * kLog2e + lg2_approx(1.0f + ex2_approx(-fabsf(x) * kLog2e));
 }
 
 // one fp32 value into three bf16 terms (hi + mid + lo carries 24 bits)
@@ -153,7 +169,7 @@ __global__ void __launch_bounds__(KdaTC::NT, 1) kda_chunk_tc(const StepParams p)
   };
   auto wait_mma = [&]() -> bool { return wait_on(&bar, phase); };
 
-  const float expA2 = expf(p.A_log[hv]) * kLog2e;  // log2 units
+  const float expA = expf(p.A_log[hv]);
   const float dtb = p.dt_bias[(int64_t)hv * D + v];
   // the token inputs of chunk c into input buffer `buf` (zero past the run)
   auto issue_loads = [&](int c, int buf) {
@@ -182,6 +198,9 @@ __global__ void __launch_bounds__(KdaTC::NT, 1) kda_chunk_tc(const StepParams p)
   auto load_beta = [&](int c) {
     if (tid < C && c * C + tid < n) nb = ld_in1(p.beta, (u.tok0 + (int64_t)c * C + tid) * p.HV + hv, true);
   };
+  // P past the diagonal (s > t) is never written by the pair loop: zero once
+  for (int i = tid; i < 3 * CT::P_BYTES / 16; i += CT::NT)
+    reinterpret_cast<uint4*>(sm + CT::P3)[i] = make_uint4(0u, 0u, 0u, 0u);
   issue_loads(0, 0);
   load_beta(0);
 
@@ -229,7 +248,7 @@ __global__ void __launch_bounds__(KdaTC::NT, 1) kda_chunk_tc(const StepParams p)
 #pragma unroll
       for (int j = 0; j < C / 2; ++j) {
         const int t = (C / 2) * wg + j;
-        const float la = t < nv ? -expA2 * softplus_f(__bfloat162float(gr[t * D]) + dtb) : 0.0f;
+        const float la = t < nv ? -expA * softplus_log2(__bfloat162float(gr[t * D]) + dtb) : 0.0f;
         acc += la;
         gl[j] = acc;
       }
@@ -238,20 +257,25 @@ __global__ void __launch_bounds__(KdaTC::NT, 1) kda_chunk_tc(const StepParams p)
     __syncthreads();
     {
       const float off = wg ? s_tot[v] : 0.0f;
+      float* Al = reinterpret_cast<float*>(sm + CT::AL);
+      float prev = off;
 #pragma unroll
       for (int j = 0; j < C / 2; ++j) {
         gl[j] += off;
         Gm[((C / 2) * wg + j) * CT::GS + v] = gl[j];
+        Al[((C / 2) * wg + j) * CT::GS + v] = ex2_approx(gl[j] - prev);
+        prev = gl[j];
       }
       if (wg == 1) s_egc[v] = ex2_approx(gl[C / 2 - 1]);
     }
     __syncthreads();
 
-    // ---- the scaled rows in two bf16 terms: [K~ ; Q~] (the B operand of G1)
-    // and K^ ^T (the B operand of the update, buffer c & 1)
+    // ---- the scaled rows [K~ ; Q~] in two bf16 terms (the B operand of G1)
 #pragma unroll 1
     for (int id = tid; id < 2 * C * 16; id += CT::NT) {
-      const int row = id >> 4, piece = id & 15, t = row & (C - 1);
+      // consecutive threads take consecutive rows of one 8-channel piece, so
+      // their 16-byte stores into the K-major tile fill whole bank rows
+      const int row = id & (2 * C - 1), piece = id >> 6, t = row & (C - 1);
       const float sc = row < C ? s_ik[t] : s_iq[t];
       const uint4 w = *reinterpret_cast<const uint4*>(raw + CT::R_KQ + row * CT::RS + piece * 16);
       const float4 g0 = *reinterpret_cast<const float4*>(Gm + t * CT::GS + 8 * piece);
@@ -267,6 +291,14 @@ __global__ void __launch_bounds__(KdaTC::NT, 1) kda_chunk_tc(const StepParams p)
       *reinterpret_cast<uint4*>(sm + CT::KQT + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
       *reinterpret_cast<uint4*>(sm + CT::KQT + CT::KQT_BYTES + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
     }
+    // ---- the state: previous chunk's update done; split S0^T, decay by
+    // e^{G_C} per key channel (this warpgroup's 64 keys of row v)
+    if (c > 0 && wait_mma()) {
+      aborted = true;
+      break;
+    }
+    // K^ ^T (the B operand of the update), now that the previous update,
+    // which read the tile, is done
     {
       const float gC = Gm[(C - 1) * CT::GS + v];
       const __nv_bfloat16* kcol = reinterpret_cast<const __nv_bfloat16*>(raw + CT::R_KQ) + v;
@@ -283,17 +315,11 @@ __global__ void __launch_bounds__(KdaTC::NT, 1) kda_chunk_tc(const StepParams p)
           split2_bf16x2(x0, x1, hw[e], lw[e]);
         }
         const uint32_t off = kmajor_offset(v, 8 * t8, C);
-        *reinterpret_cast<uint4*>(sm + CT::KBT + (2 * buf) * CT::KBT_BYTES + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
-        *reinterpret_cast<uint4*>(sm + CT::KBT + (2 * buf + 1) * CT::KBT_BYTES + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+        *reinterpret_cast<uint4*>(sm + CT::KBT + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+        *reinterpret_cast<uint4*>(sm + CT::KBT + CT::KBT_BYTES + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
       }
     }
 
-    // ---- the state: previous chunk's update done; split S0^T, decay by
-    // e^{G_C} per key channel (this warpgroup's 64 keys of row v)
-    if (c > 0 && wait_mma()) {
-      aborted = true;
-      break;
-    }
 #pragma unroll 1
     for (int kk = 0; kk < 2; ++kk) {
       const int kc = 2 * wg + kk;
@@ -349,52 +375,78 @@ __global__ void __launch_bounds__(KdaTC::NT, 1) kda_chunk_tc(const StepParams p)
       umma_commit(&bar);
     }
 
-    // ---- A and P on the CUDA cores while G1 runs: thread (t, sg) takes the
-    // pairs (t, s) with s = sg, sg + 8, sg + 16, sg + 24 and s <= t, over all
-    // key channels, one exponential per pair and channel
+    // ---- A and P on the CUDA cores while G1 runs. The pairs (t, s <= t) of
+    // row t come in groups of up to three consecutive s; the 187 groups of
+    // the chunk are spread over the eight warps (group 8 l + w to lane l of
+    // warp w). A group takes e^{G_t - G_s} at its largest s with one
+    // exponential per key channel and steps down with
+    // e^{G_t - G_(s-1)} = e^{G_t - G_s} alpha_s (every factor <= 1), so a
+    // chunk needs about a third of the exponentials of one per pair.
+    // Channels are taken in pairs with the paired fp32 instructions.
     {
-      const int t = tid >> 3, sg = tid & 7;
-      const int nj = t >= sg ? min(3, (t - sg) >> 3) + 1 : 0;
-      float a[4] = {0.f, 0.f, 0.f, 0.f}, pq[4] = {0.f, 0.f, 0.f, 0.f};
-      const unsigned char* krow = raw + CT::R_KQ;
-#pragma unroll 2
-      for (int i4 = 0; i4 < D; i4 += 4) {
-        const float4 gt = *reinterpret_cast<const float4*>(Gm + t * CT::GS + i4);
-        const uint2 kw = *reinterpret_cast<const uint2*>(krow + t * CT::RS + i4 * 2);
-        const uint2 qw = *reinterpret_cast<const uint2*>(krow + (C + t) * CT::RS + i4 * 2);
-        const float kt[4] = {bf16_lo(kw.x), bf16_hi(kw.x), bf16_lo(kw.y), bf16_hi(kw.y)};
-        const float qt[4] = {bf16_lo(qw.x), bf16_hi(qw.x), bf16_lo(qw.y), bf16_hi(qw.y)};
-        const float gtv[4] = {gt.x, gt.y, gt.z, gt.w};
+      const int item = 8 * (tid & 31) + (tid >> 5);
+      int t = 0, rem = item;
+      while (t < C && rem >= (t + 3) / 3) {
+        rem -= (t + 3) / 3;
+        ++t;
+      }
+      if (t < C) {
+        const int s0 = 3 * rem;
+        const int shi = min(s0 + 2, t);  // pairs shi, shi - 1, shi - 2 (those >= s0 are kept)
+        const int sm1 = max(shi - 1, 0), sm2 = max(shi - 2, 0);
+        const float* Al = reinterpret_cast<const float*>(sm + CT::AL);
+        float2 a2[3], p2[3];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          if (j < nj) {
-            const int s = sg + 8 * j;
-            const float4 gs = *reinterpret_cast<const float4*>(Gm + s * CT::GS + i4);
-            const uint2 sw = *reinterpret_cast<const uint2*>(krow + s * CT::RS + i4 * 2);
-            const float ks[4] = {bf16_lo(sw.x), bf16_hi(sw.x), bf16_lo(sw.y), bf16_hi(sw.y)};
-            const float gsv[4] = {gs.x, gs.y, gs.z, gs.w};
+        for (int j = 0; j < 3; ++j) a2[j] = p2[j] = make_float2(0.f, 0.f);
+        const unsigned char* krow = raw + CT::R_KQ;
+#pragma unroll 4
+        for (int i4 = 0; i4 < D; i4 += 4) {
+          const float4 gt = *reinterpret_cast<const float4*>(Gm + t * CT::GS + i4);
+          const float4 gs = *reinterpret_cast<const float4*>(Gm + shi * CT::GS + i4);
+          const float4 al0 = *reinterpret_cast<const float4*>(Al + shi * CT::GS + i4);
+          const float4 al1 = *reinterpret_cast<const float4*>(Al + sm1 * CT::GS + i4);
+          const uint2 kw = *reinterpret_cast<const uint2*>(krow + t * CT::RS + i4 * 2);
+          const uint2 qw = *reinterpret_cast<const uint2*>(krow + (C + t) * CT::RS + i4 * 2);
+          const uint2 sw[3] = {*reinterpret_cast<const uint2*>(krow + shi * CT::RS + i4 * 2),
+                               *reinterpret_cast<const uint2*>(krow + sm1 * CT::RS + i4 * 2),
+                               *reinterpret_cast<const uint2*>(krow + sm2 * CT::RS + i4 * 2)};
+          const float2 kt0 = make_float2(bf16_lo(kw.x), bf16_hi(kw.x)), kt1 = make_float2(bf16_lo(kw.y), bf16_hi(kw.y));
+          const float2 qt0 = make_float2(bf16_lo(qw.x), bf16_hi(qw.x)), qt1 = make_float2(bf16_lo(qw.y), bf16_hi(qw.y));
+          const float2 d0 = __fadd2_rn(make_float2(gt.x, gt.y), make_float2(-gs.x, -gs.y));
+          const float2 d1 = __fadd2_rn(make_float2(gt.z, gt.w), make_float2(-gs.z, -gs.w));
+          float2 e0 = make_float2(ex2_approx(d0.x), ex2_approx(d0.y));
+          float2 e1 = make_float2(ex2_approx(d1.x), ex2_approx(d1.y));
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const float w = ks[e] * ex2_approx(gtv[e] - gsv[e]);
-              a[j] = fmaf(kt[e], w, a[j]);
-              pq[j] = fmaf(qt[e], w, pq[j]);
+          for (int j = 0; j < 3; ++j) {
+            const float2 w0 = __fmul2_rn(make_float2(bf16_lo(sw[j].x), bf16_hi(sw[j].x)), e0);
+            const float2 w1 = __fmul2_rn(make_float2(bf16_lo(sw[j].y), bf16_hi(sw[j].y)), e1);
+            a2[j] = __ffma2_rn(kt0, w0, a2[j]);
+            a2[j] = __ffma2_rn(kt1, w1, a2[j]);
+            p2[j] = __ffma2_rn(qt0, w0, p2[j]);
+            p2[j] = __ffma2_rn(qt1, w1, p2[j]);
+            if (j == 0) {
+              e0 = __fmul2_rn(e0, make_float2(al0.x, al0.y));
+              e1 = __fmul2_rn(e1, make_float2(al0.z, al0.w));
+            } else if (j == 1) {
+              e0 = __fmul2_rn(e0, make_float2(al1.x, al1.y));
+              e1 = __fmul2_rn(e1, make_float2(al1.z, al1.w));
             }
           }
         }
-      }
-      float* arow = reinterpret_cast<float*>(sm + CT::AM) + t * CT::AS;
+        float* arow = reinterpret_cast<float*>(sm + CT::AM) + t * CT::AS;
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const int s = sg + 8 * j;
-        const float av = s < t ? s_beta[t] * s_ik[t] * s_ik[s] * a[j] : 0.0f;
-        const float pv = s <= t ? s_iq[t] * s_ik[s] * pq[j] : 0.0f;
-        arow[s] = av;
-        uint16_t ph, pm, pl;
-        split3_bf16(pv, ph, pm, pl);
-        const uint32_t off = kmajor_offset(t, s, C);
-        *reinterpret_cast<uint16_t*>(sm + CT::P3 + off) = ph;
-        *reinterpret_cast<uint16_t*>(sm + CT::P3 + CT::P_BYTES + off) = pm;
-        *reinterpret_cast<uint16_t*>(sm + CT::P3 + 2 * CT::P_BYTES + off) = pl;
+        for (int j = 0; j < 3; ++j) {
+          const int sx = shi - j;
+          if (sx >= s0) {
+            arow[sx] = sx < t ? s_beta[t] * s_ik[t] * s_ik[sx] * (a2[j].x + a2[j].y) : 0.0f;
+            uint16_t ph, pm, pl;
+            split3_bf16(s_iq[t] * s_ik[sx] * (p2[j].x + p2[j].y), ph, pm, pl);
+            const uint32_t off = kmajor_offset(t, sx, C);
+            *reinterpret_cast<uint16_t*>(sm + CT::P3 + off) = ph;
+            *reinterpret_cast<uint16_t*>(sm + CT::P3 + CT::P_BYTES + off) = pm;
+            *reinterpret_cast<uint16_t*>(sm + CT::P3 + 2 * CT::P_BYTES + off) = pl;
+          }
+        }
       }
     }
     if (wait_mma()) {  // G1; also orders A and P before the reads below
@@ -501,7 +553,7 @@ __global__ void __launch_bounds__(KdaTC::NT, 1) kda_chunk_tc(const StepParams p)
 #pragma unroll 1
           for (int ks = 0; ks < C / 16; ++ks)
             umma_bf16(tmem + CT::T_ST, umma_desc_kmajor(sm + CT::UT3 + i * CT::UT_BYTES + ks * 256, C),
-                      umma_desc_kmajor(sm + CT::KBT + (2 * buf + j) * CT::KBT_BYTES + ks * 256, C), id_up, true);
+                      umma_desc_kmajor(sm + CT::KBT + j * CT::KBT_BYTES + ks * 256, C), id_up, true);
       umma_commit(&bar);
     }
     if (wait_on(&bar_o, phase_o)) {
