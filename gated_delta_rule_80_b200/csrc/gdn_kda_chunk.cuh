@@ -376,15 +376,15 @@ __global__ void __launch_bounds__(KdaTC::NT, 1) kda_chunk_tc(const StepParams p)
     }
 
     // ---- A and P on the CUDA cores while G1 runs. The pairs (t, s <= t) of
-    // row t come in groups of up to three consecutive s; the 187 groups of
-    // the chunk are spread over the eight warps (group 8 l + w to lane l of
-    // warp w). A group takes e^{G_t - G_s} at its largest s with one
+    // row t come in groups of up to three consecutive s; group g goes to
+    // thread g (187 groups), so the lanes of a warp share few t-rows and
+    // their t-row loads broadcast. A group takes e^{G_t - G_s} at its largest s with one
     // exponential per key channel and steps down with
     // e^{G_t - G_(s-1)} = e^{G_t - G_s} alpha_s (every factor <= 1), so a
     // chunk needs about a third of the exponentials of one per pair.
     // Channels are taken in pairs with the paired fp32 instructions.
     {
-      const int item = 8 * (tid & 31) + (tid >> 5);
+      const int item = tid;
       int t = 0, rem = item;
       while (t < C && rem >= (t + 3) / 3) {
         rem -= (t + 3) / 3;
