@@ -222,12 +222,11 @@ __global__ void __launch_bounds__(ChunkTC::NT, 1) prefill_chunk_tc(const StepPar
     // chunk's rows, so it runs under the prologue and the state split
     if (tid == 0) {
       tc_fence_after_sync();
-      const unsigned char* kq0 = sm + CT::KQ + buf * CT::KQ_BYTES;
+      const uint64_t dk = umma_desc_kmajor(sm + CT::KQ + buf * CT::KQ_BYTES, D);
       const uint32_t id_gr = umma_idesc_bf16(128, 64);
-#pragma unroll 1
+#pragma unroll
       for (int ks = 0; ks < D / 16; ++ks)
-        umma_bf16(tmem + CT::T_GR, umma_desc_kmajor(kq0 + ks * 256, D), umma_desc_kmajor(kq0 + ks * 256, D), id_gr,
-                  ks > 0);
+        umma_bf16(tmem + CT::T_GR, umma_desc_add(dk, ks * 256), umma_desc_add(dk, ks * 256), id_gr, ks > 0);
       umma_commit(&bar_gr);
     }
     if (c + 1 < nchunks) {
@@ -299,43 +298,60 @@ __global__ void __launch_bounds__(ChunkTC::NT, 1) prefill_chunk_tc(const StepPar
         if (tid == 0) raise_err(p.err, E_PAGE_RANGE);
         snap = -1;
       }
-#pragma unroll 1
-      for (int kk = 0; kk < 2; ++kk) {
-        const int kc = 2 * wg + kk;
-        float x[32];
-        if (c == 0) {
+      // both 32-column blocks of this warpgroup's half of row v are loaded
+      // (and stored back) with one wait for the pair
+      float x[2][32];
+      if (c == 0) {
+#pragma unroll
+        for (int kk = 0; kk < 2; ++kk) {
+          const int kc = 2 * wg + kk;
           if (u.fresh) {
 #pragma unroll
-            for (int i = 0; i < 32; ++i) x[i] = 0.0f;
+            for (int i = 0; i < 32; ++i) x[kk][i] = 0.0f;
           } else {
             const float4* src = reinterpret_cast<const float4*>(pool + (u.src * p.HV + hv) * head + (int64_t)v * D + 32 * kc);
 #pragma unroll
             for (int q = 0; q < 8; ++q) {
               const float4 f = __ldcs(src + q);
-              x[4 * q] = f.x; x[4 * q + 1] = f.y; x[4 * q + 2] = f.z; x[4 * q + 3] = f.w;
+              x[kk][4 * q] = f.x; x[kk][4 * q + 1] = f.y; x[kk][4 * q + 2] = f.z; x[kk][4 * q + 3] = f.w;
             }
           }
-        } else {
-          tmem_ld32(t_st + 32 * kc, x);
         }
+      } else {
+        uint32_t r0[32], r1[32];
+        tmem_ld32_issue(t_st + 64 * wg, r0);
+        tmem_ld32_issue(t_st + 64 * wg + 32, r1);
+        tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          x[0][i] = __uint_as_float(r0[i]);
+          x[1][i] = __uint_as_float(r1[i]);
+        }
+      }
+#pragma unroll
+      for (int kk = 0; kk < 2; ++kk) {
+        const int kc = 2 * wg + kk;
         if (snap >= 0) {
           float4* dst = reinterpret_cast<float4*>(pool + (snap * p.HV + hv) * head + (int64_t)v * D + 32 * kc);
 #pragma unroll
-          for (int q = 0; q < 8; ++q) __stcs(dst + q, make_float4(x[4 * q], x[4 * q + 1], x[4 * q + 2], x[4 * q + 3]));
+          for (int q = 0; q < 8; ++q)
+            __stcs(dst + q, make_float4(x[kk][4 * q], x[kk][4 * q + 1], x[kk][4 * q + 2], x[kk][4 * q + 3]));
         }
 #pragma unroll
         for (int q8 = 0; q8 < 4; ++q8) {
           uint32_t hw[4], lw[4];
 #pragma unroll
-          for (int i = 0; i < 4; ++i) split2_bf16x2(x[8 * q8 + 2 * i], x[8 * q8 + 2 * i + 1], hw[i], lw[i]);
+          for (int i = 0; i < 4; ++i) split2_bf16x2(x[kk][8 * q8 + 2 * i], x[kk][8 * q8 + 2 * i + 1], hw[i], lw[i]);
           const uint32_t off = kmajor_offset(v, 32 * kc + 8 * q8, D);
           *reinterpret_cast<uint4*>(sm + CT::S3 + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
           *reinterpret_cast<uint4*>(sm + CT::S3 + CT::S3_BYTES + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
         }
 #pragma unroll
-        for (int i = 0; i < 32; ++i) x[i] *= eC;
-        tmem_st32(t_st + 32 * kc, x);
+        for (int i = 0; i < 32; ++i) x[kk][i] *= eC;
       }
+      tmem_st32_issue(t_st + 64 * wg, x[0]);
+      tmem_st32_issue(t_st + 64 * wg + 32, x[1]);
+      tmem_wait_st();
     }
     fence_async_smem();
     tc_fence_before_sync();
@@ -345,12 +361,13 @@ __global__ void __launch_bounds__(ChunkTC::NT, 1) prefill_chunk_tc(const StepPar
     if (tid == 0) {
       tc_fence_after_sync();
       const uint32_t id_g1 = umma_idesc_bf16(128, 128);
-#pragma unroll 1
+      const uint64_t da = umma_desc_kmajor(sm + CT::S3, D), db = umma_desc_kmajor(kq, D);
+#pragma unroll
       for (int i = 0; i < 2; ++i)
-#pragma unroll 1
+#pragma unroll
         for (int ks = 0; ks < D / 16; ++ks)
-          umma_bf16(tmem + CT::T_G1, umma_desc_kmajor(sm + CT::S3 + i * CT::S3_BYTES + ks * 256, D),
-                    umma_desc_kmajor(kq + ks * 256, D), id_g1, i > 0 || ks > 0);
+          umma_bf16(tmem + CT::T_G1, umma_desc_add(da, i * CT::S3_BYTES + ks * 256), umma_desc_add(db, ks * 256), id_g1,
+                    i > 0 || ks > 0);
       umma_commit(&bar);
     }
     // the Gram (issued first): A, P and K^T do not wait for G1
@@ -524,17 +541,15 @@ __global__ void __launch_bounds__(ChunkTC::NT, 1) prefill_chunk_tc(const StepPar
     if (tid == 0) {
       tc_fence_after_sync();
       const uint32_t id_o = umma_idesc_bf16(128, 64);
-      bool acc = false;
-#pragma unroll 1
+      const uint64_t da = umma_desc_kmajor(sm + CT::UT3, C), db = umma_desc_kmajor(sm + CT::P3, C);
+#pragma unroll
       for (int i = 0; i < 3; ++i)
-#pragma unroll 1
+#pragma unroll
         for (int j = 0; i + j < 3; ++j)
-#pragma unroll 1
-          for (int ks = 0; ks < C / 16; ++ks) {
-            umma_bf16(tmem + CT::T_GR, umma_desc_kmajor(sm + CT::UT3 + i * CT::UT_BYTES + ks * 256, C),
-                      umma_desc_kmajor(sm + CT::P3 + j * CT::P_BYTES + ks * 256, C), id_o, acc);
-            acc = true;
-          }
+#pragma unroll
+          for (int ks = 0; ks < C / 16; ++ks)
+            umma_bf16(tmem + CT::T_GR, umma_desc_add(da, i * CT::UT_BYTES + ks * 256),
+                      umma_desc_add(db, j * CT::P_BYTES + ks * 256), id_o, i + j + ks > 0);
       umma_commit(&bar_gr);
     }
     if (wait_on(&bar_gr, phase_gr)) {
@@ -599,12 +614,13 @@ __global__ void __launch_bounds__(ChunkTC::NT, 1) prefill_chunk_tc(const StepPar
     if (tid == 0) {
       tc_fence_after_sync();
       const uint32_t id_up = umma_idesc_bf16(128, 128);
-#pragma unroll 1
+      const uint64_t da = umma_desc_kmajor(sm + CT::UT3, C), db = umma_desc_kmajor(sm + CT::KT, C);
+#pragma unroll
       for (int i = 0; i < 3; ++i)
-#pragma unroll 1
+#pragma unroll
         for (int ks = 0; ks < C / 16; ++ks)
-          umma_bf16(tmem + CT::T_ST, umma_desc_kmajor(sm + CT::UT3 + i * CT::UT_BYTES + ks * 256, C),
-                    umma_desc_kmajor(sm + CT::KT + ks * 256, C), id_up, true);
+          umma_bf16(tmem + CT::T_ST, umma_desc_add(da, i * CT::UT_BYTES + ks * 256), umma_desc_add(db, ks * 256), id_up,
+                    true);
       umma_commit(&bar);
     }
   }

@@ -320,37 +320,55 @@ __global__ void __launch_bounds__(KdaTC::NT, 1) kda_chunk_tc(const StepParams p)
       }
     }
 
-#pragma unroll 1
-    for (int kk = 0; kk < 2; ++kk) {
-      const int kc = 2 * wg + kk;
-      float x[32];
+    {
+      // both 32-key blocks of this warpgroup's half of row v are loaded (and
+      // stored back) with one wait for the pair
+      float x[2][32];
       if (c == 0) {
-        if constexpr (L == L_VFIRST) {
-          const float4* src = reinterpret_cast<const float4*>(state + (int64_t)v * D + 32 * kc);
 #pragma unroll
-          for (int q = 0; q < 8; ++q) {
-            const float4 f = __ldcs(src + q);
-            x[4 * q] = f.x; x[4 * q + 1] = f.y; x[4 * q + 2] = f.z; x[4 * q + 3] = f.w;
+        for (int kk = 0; kk < 2; ++kk) {
+          const int kc = 2 * wg + kk;
+          if constexpr (L == L_VFIRST) {
+            const float4* src = reinterpret_cast<const float4*>(state + (int64_t)v * D + 32 * kc);
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+              const float4 f = __ldcs(src + q);
+              x[kk][4 * q] = f.x; x[kk][4 * q + 1] = f.y; x[kk][4 * q + 2] = f.z; x[kk][4 * q + 3] = f.w;
+            }
+          } else {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) x[kk][j] = __ldcs(state + (int64_t)(32 * kc + j) * D + v);
           }
-        } else {
-#pragma unroll
-          for (int j = 0; j < 32; ++j) x[j] = __ldcs(state + (int64_t)(32 * kc + j) * D + v);
         }
       } else {
-        tmem_ld32(t_st + 32 * kc, x);
+        uint32_t r0[32], r1[32];
+        tmem_ld32_issue(t_st + 64 * wg, r0);
+        tmem_ld32_issue(t_st + 64 * wg + 32, r1);
+        tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          x[0][i] = __uint_as_float(r0[i]);
+          x[1][i] = __uint_as_float(r1[i]);
+        }
       }
 #pragma unroll
-      for (int q8 = 0; q8 < 4; ++q8) {
-        uint32_t hw[4], lw[4];
+      for (int kk = 0; kk < 2; ++kk) {
+        const int kc = 2 * wg + kk;
 #pragma unroll
-        for (int i = 0; i < 4; ++i) split2_bf16x2(x[8 * q8 + 2 * i], x[8 * q8 + 2 * i + 1], hw[i], lw[i]);
-        const uint32_t off = kmajor_offset(v, 32 * kc + 8 * q8, D);
-        *reinterpret_cast<uint4*>(sm + CT::X + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
-        *reinterpret_cast<uint4*>(sm + CT::X + CT::S_BYTES + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+        for (int q8 = 0; q8 < 4; ++q8) {
+          uint32_t hw[4], lw[4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) split2_bf16x2(x[kk][8 * q8 + 2 * i], x[kk][8 * q8 + 2 * i + 1], hw[i], lw[i]);
+          const uint32_t off = kmajor_offset(v, 32 * kc + 8 * q8, D);
+          *reinterpret_cast<uint4*>(sm + CT::X + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+          *reinterpret_cast<uint4*>(sm + CT::X + CT::S_BYTES + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+        }
+#pragma unroll
+        for (int i = 0; i < 32; ++i) x[kk][i] *= s_egc[32 * kc + i];
       }
-#pragma unroll
-      for (int i = 0; i < 32; ++i) x[i] *= s_egc[32 * kc + i];
-      tmem_st32(t_st + 32 * kc, x);
+      tmem_st32_issue(t_st + 64 * wg, x[0]);
+      tmem_st32_issue(t_st + 64 * wg + 32, x[1]);
+      tmem_wait_st();
     }
     fence_async_smem();
     tc_fence_before_sync();
@@ -361,16 +379,14 @@ __global__ void __launch_bounds__(KdaTC::NT, 1) kda_chunk_tc(const StepParams p)
     if (tid == 0) {
       tc_fence_after_sync();
       const uint32_t id_g1 = umma_idesc_bf16(128, 2 * C);
-      bool acc = false;
-#pragma unroll 1
+      const uint64_t da = umma_desc_kmajor(sm + CT::X, D), db = umma_desc_kmajor(sm + CT::KQT, D);
+#pragma unroll
       for (int ij = 0; ij < 3; ++ij) {
         const int i = ij == 2 ? 1 : 0, j = ij == 1 ? 1 : 0;
-#pragma unroll 1
-        for (int ks = 0; ks < D / 16; ++ks) {
-          umma_bf16(tmem + CT::T_G1, umma_desc_kmajor(sm + CT::X + i * CT::S_BYTES + ks * 256, D),
-                    umma_desc_kmajor(sm + CT::KQT + j * CT::KQT_BYTES + ks * 256, D), id_g1, acc);
-          acc = true;
-        }
+#pragma unroll
+        for (int ks = 0; ks < D / 16; ++ks)
+          umma_bf16(tmem + CT::T_G1, umma_desc_add(da, i * CT::S_BYTES + ks * 256),
+                    umma_desc_add(db, j * CT::KQT_BYTES + ks * 256), id_g1, ij + ks > 0);
       }
       umma_commit(&bar);
     }
@@ -533,27 +549,26 @@ __global__ void __launch_bounds__(KdaTC::NT, 1) kda_chunk_tc(const StepParams p)
     if (tid == 0) {
       tc_fence_after_sync();
       const uint32_t id_o = umma_idesc_bf16(128, C);
-      bool acc = false;
-#pragma unroll 1
+      const uint64_t du = umma_desc_kmajor(sm + CT::UT3, C), dp = umma_desc_kmajor(sm + CT::P3, C);
+#pragma unroll
       for (int i = 0; i < 3; ++i)
-#pragma unroll 1
+#pragma unroll
         for (int j = 0; i + j < 3; ++j)
-#pragma unroll 1
-          for (int ks = 0; ks < C / 16; ++ks) {
-            umma_bf16(tmem + CT::T_O, umma_desc_kmajor(sm + CT::UT3 + i * CT::UT_BYTES + ks * 256, C),
-                      umma_desc_kmajor(sm + CT::P3 + j * CT::P_BYTES + ks * 256, C), id_o, acc);
-            acc = true;
-          }
+#pragma unroll
+          for (int ks = 0; ks < C / 16; ++ks)
+            umma_bf16(tmem + CT::T_O, umma_desc_add(du, i * CT::UT_BYTES + ks * 256),
+                      umma_desc_add(dp, j * CT::P_BYTES + ks * 256), id_o, i + j + ks > 0);
       umma_commit(&bar_o);
       const uint32_t id_up = umma_idesc_bf16(128, D);
-#pragma unroll 1
+      const uint64_t dk = umma_desc_kmajor(sm + CT::KBT, C);
+#pragma unroll
       for (int i = 0; i < 3; ++i)
-#pragma unroll 1
+#pragma unroll
         for (int j = 0; j < 2 && i + j < 3; ++j)
-#pragma unroll 1
+#pragma unroll
           for (int ks = 0; ks < C / 16; ++ks)
-            umma_bf16(tmem + CT::T_ST, umma_desc_kmajor(sm + CT::UT3 + i * CT::UT_BYTES + ks * 256, C),
-                      umma_desc_kmajor(sm + CT::KBT + j * CT::KBT_BYTES + ks * 256, C), id_up, true);
+            umma_bf16(tmem + CT::T_ST, umma_desc_add(du, i * CT::UT_BYTES + ks * 256),
+                      umma_desc_add(dk, j * CT::KBT_BYTES + ks * 256), id_up, true);
       umma_commit(&bar);
     }
     if (wait_on(&bar_o, phase_o)) {
