@@ -61,8 +61,14 @@ struct ChunkTC {
   static constexpr uint32_t KT = UT3 + 3 * UT_BYTES;  // [128 x 64] bf16, K-major: K^T
   static constexpr uint32_t P3 = KT + UT_BYTES;       // 3 x [64 x 64] bf16, K-major: P split
   static constexpr uint32_t P_BYTES = C * C * 2;
-  static constexpr uint32_t SMEM = S3 + 3 * S3_BYTES;
-  static_assert(AM + C * AS * 4 <= KT && P3 + 3 * P_BYTES <= SMEM, "chunk operands fit in the S3 region");
+  // the update operand (diag(w) U)^T in two bf16 terms (16 bits: the state
+  // moves by about 5e-6), written beside U^T so that the output product and
+  // the update are issued together
+  // (starting in the S3 region's unused tail, after P)
+  static constexpr uint32_t WU2 = P3 + 3 * P_BYTES;  // 2 x [128 x 64] bf16, K-major
+  static constexpr uint32_t SMEM = WU2 + 2 * UT_BYTES;
+  static_assert(AM + C * AS * 4 <= KT && SMEM >= S3 + 3 * S3_BYTES, "chunk operands fit in the S3 region");
+  static_assert(SMEM + 4096 <= 227 * 1024, "dynamic plus static shared memory within one CTA's 227 KiB");
   // tensor memory columns
   static constexpr uint32_t T_ST = 0, T_G1 = 128, T_GR = 256, T_COLS = 512;
 };
@@ -534,6 +540,13 @@ __global__ void __launch_bounds__(ChunkTC::NT, 1) prefill_chunk_tc(const StepPar
       *reinterpret_cast<uint4*>(sm + CT::UT3 + off) = hh;
       *reinterpret_cast<uint4*>(sm + CT::UT3 + CT::UT_BYTES + off) = mm;
       *reinterpret_cast<uint4*>(sm + CT::UT3 + 2 * CT::UT_BYTES + off) = ll;
+      // the update operand (diag(w) U)^T, two terms
+      uint32_t hw[4], lw[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        split2_bf16x2(s_wc[8 * t8 + 2 * i] * x[2 * i], s_wc[8 * t8 + 2 * i + 1] * x[2 * i + 1], hw[i], lw[i]);
+      *reinterpret_cast<uint4*>(sm + CT::WU2 + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+      *reinterpret_cast<uint4*>(sm + CT::WU2 + CT::UT_BYTES + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
     }
     fence_async_smem();
     tc_fence_before_sync();
@@ -551,6 +564,17 @@ __global__ void __launch_bounds__(ChunkTC::NT, 1) prefill_chunk_tc(const StepPar
             umma_bf16(tmem + CT::T_GR, umma_desc_add(da, i * CT::UT_BYTES + ks * 256),
                       umma_desc_add(db, j * CT::P_BYTES + ks * 256), id_o, i + j + ks > 0);
       umma_commit(&bar_gr);
+      // ---- S^T += (diag(w) U)^T K on the tensor cores (the state was decayed
+      // above); it completes while the outputs are stored
+      const uint32_t id_up = umma_idesc_bf16(128, 128);
+      const uint64_t dw = umma_desc_kmajor(sm + CT::WU2, C), dkt = umma_desc_kmajor(sm + CT::KT, C);
+#pragma unroll
+      for (int i = 0; i < 2; ++i)
+#pragma unroll
+        for (int ks = 0; ks < C / 16; ++ks)
+          umma_bf16(tmem + CT::T_ST, umma_desc_add(dw, i * CT::UT_BYTES + ks * 256), umma_desc_add(dkt, ks * 256), id_up,
+                    true);
+      umma_commit(&bar);
     }
     if (wait_on(&bar_gr, phase_gr)) {
       aborted = true;
@@ -579,28 +603,9 @@ __global__ void __launch_bounds__(ChunkTC::NT, 1) prefill_chunk_tc(const StepPar
         }
       }
     }
-    // ---- update operand (diag(w) U)^T, split in three bf16 terms (tokens 32 wg ..)
-#pragma unroll 1
-    for (int tt = 0; tt < 4; ++tt) {
-      const int t8 = 4 * wg + tt;
-      float x[8];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const int t = 8 * t8 + i;
-        x[i] = s_wc[t] * Us[t * D + v];
-      }
-      uint4 hh, mm, ll;
-      split3_bf16x8(x, hh, mm, ll);
-      const uint32_t off = kmajor_offset(v, 8 * t8, C);
-      *reinterpret_cast<uint4*>(sm + CT::UT3 + off) = hh;
-      *reinterpret_cast<uint4*>(sm + CT::UT3 + CT::UT_BYTES + off) = mm;
-      *reinterpret_cast<uint4*>(sm + CT::UT3 + 2 * CT::UT_BYTES + off) = ll;
-    }
-    fence_async_smem();
-    tc_fence_before_sync();
-    __syncthreads();
     if (out_bf16) {
       // the staged bf16 outputs: 16 bytes (8 values of one token) per copy
+      __syncthreads();
       const uint4* ost = reinterpret_cast<const uint4*>(sm + CT::VB + buf * CT::V_BYTES);
 #pragma unroll
       for (int k = 0; k < C * D / 8 / CT::NT; ++k) {
@@ -609,19 +614,6 @@ __global__ void __launch_bounds__(ChunkTC::NT, 1) prefill_chunk_tc(const StepPar
         if (pos >= pos_lo && pos < pos_hi)
           __stcs(reinterpret_cast<uint4*>(p.out) + ((u.tok0 + (pos - pos_lo)) * p.HV + hv) * (D / 8) + piece, ost[id]);
       }
-    }
-    // ---- S^T += (diag(w) U)^T K on the tensor cores (the state was decayed above)
-    if (tid == 0) {
-      tc_fence_after_sync();
-      const uint32_t id_up = umma_idesc_bf16(128, 128);
-      const uint64_t da = umma_desc_kmajor(sm + CT::UT3, C), db = umma_desc_kmajor(sm + CT::KT, C);
-#pragma unroll
-      for (int i = 0; i < 3; ++i)
-#pragma unroll
-        for (int ks = 0; ks < C / 16; ++ks)
-          umma_bf16(tmem + CT::T_ST, umma_desc_add(da, i * CT::UT_BYTES + ks * 256), umma_desc_add(db, ks * 256), id_up,
-                    true);
-      umma_commit(&bar);
     }
   }
 

@@ -69,6 +69,7 @@ struct KdaTC {
   static constexpr uint32_t UT_BYTES = D * C * 2;
   static constexpr uint32_t SMEM = X + 2 * S_BYTES;
   static_assert(UT3 + 3 * UT_BYTES <= SMEM, "U and its split fit where the S0 split was");
+  static_assert(SMEM + 2048 <= 227 * 1024, "dynamic plus static shared memory within one CTA's 227 KiB");
   static_assert(KQT % 16 == 0 && KBT % 16 == 0 && AL % 16 == 0 && P3 % 16 == 0 && X % 16 == 0 && UT3 % 16 == 0,
                 "16-byte tiles");
   // tensor memory columns: state, G1 (32 k columns then 32 q columns), O
