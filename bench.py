@@ -18,6 +18,7 @@ collective); timing is the max over ranks.
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import hashlib
 import json
 import math
@@ -60,6 +61,10 @@ def parse():
     ap.add_argument("--seconds", type=float, default=1.0,
                     help="device time each timed configuration covers (repetitions of --steps steps)")
     ap.add_argument("--headline-only", action="store_true", help="skip the by_config entries")
+    ap.add_argument("--batch", type=int, default=0,
+                    help="sequences of the headline workload (default: the workload's own); a smaller batch keeps "
+                         "a profiler capture of the paged pool to a few GB")
+    ap.add_argument("--warm-seconds", type=float, default=0.3, help="clock warm-up before each timed configuration")
     return ap.parse_args()
 
 
@@ -480,8 +485,10 @@ class PrefillRun:
                 f"H={self.H}, HV={self.HV}, K=V={self.K}, bf16 in/out, fp32 pages (one snapshot per page)")
 
 
-def make_run(name, rank, layout=None):
+def make_run(name, rank, layout=None, batch=0):
     w = W.WORKLOADS.get(name)
+    if batch and w is not None:
+        w = dataclasses.replace(w, B=batch)
     if name in ("slots", "fp8", "int8", "tiny"):
         return SlotsRun(w, rank)
     if name == "paged":
@@ -611,13 +618,13 @@ def capture(run, n):
     return g
 
 
-def time_steps(run, K, warmup, world, local, min_seconds):
+def time_steps(run, K, warmup, world, local, min_seconds, warm_seconds=0.3):
     """Times exactly K steps per repetition, repeated until min_seconds of
     device time are covered (at least MIN_REPS repetitions), with NVML
     sampling the clocks over the whole window. Returns the median
     repetition's milliseconds (max over ranks), all repetitions, and the
     clock summary."""
-    t_end = time.perf_counter() + 0.3          # clocks up, kernels loaded
+    t_end = time.perf_counter() + warm_seconds  # clocks up, kernels loaded
     i = 0
     while time.perf_counter() < t_end:
         for _ in range(20):
@@ -673,9 +680,9 @@ def run_b200(args, world, rank, local):
     G.lib()
     K = args.steps
     peak, peak_kind = measured_peak()
-    run = make_run(args.workload, rank)
+    run = make_run(args.workload, rank, batch=args.batch)
     desc, tps, l2 = run.describe(), run.tokens_per_step, run.l2_note
-    tm = time_steps(run, K, args.warmup, world, local, args.seconds)
+    tm = time_steps(run, K, args.warmup, world, local, args.seconds, args.warm_seconds)
     total_ms = tm["median_ms"]
     value = world * run.tokens_per_step * K / (total_ms / 1e3)
     ms_per_step = total_ms / K
@@ -725,7 +732,7 @@ def run_b200(args, world, rank, local):
     if not args.headline_only:
         for name, wl, kw in BY_CONFIG:
             r = make_run(wl, rank, **kw)
-            t = time_steps(r, K, args.warmup, world, local, args.seconds)
+            t = time_steps(r, K, args.warmup, world, local, args.seconds, args.warm_seconds)
             us = t["median_ms"] * 1e3 / K
             entry = {"workload": r.describe(), "us_per_launch": us,
                      "tokens_per_s": world * r.tokens_per_step * K / (t["median_ms"] / 1e3),
