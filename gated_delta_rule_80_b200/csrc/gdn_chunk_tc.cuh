@@ -70,7 +70,11 @@ struct ChunkTC {
   static_assert(AM + C * AS * 4 <= KT && SMEM >= S3 + 3 * S3_BYTES, "chunk operands fit in the S3 region");
   static_assert(SMEM + 4096 <= 227 * 1024, "dynamic plus static shared memory within one CTA's 227 KiB");
   // tensor memory columns
-  static constexpr uint32_t T_ST = 0, T_G1 = 128, T_GR = 256, T_COLS = 512;
+  // tensor memory columns: state, G1, Gram / outputs, and the page snapshot
+  // of the chunk's initial state, stored to the pool a quarter at a time
+  // over the chunk instead of in one burst (every CTA writing 64 KiB at the
+  // same point stalled its warps on the stores)
+  static constexpr uint32_t T_ST = 0, T_G1 = 128, T_GR = 256, T_SN = 320, T_COLS = 512;
 };
 
 // Splits of fp32 pairs into bf16 terms with the paired hardware conversion
@@ -188,6 +192,7 @@ __global__ void __launch_bounds__(ChunkTC::NT, 1) prefill_chunk_tc(const StepPar
   const uint32_t t_st = tmem + CT::T_ST + lane_base;
   const uint32_t t_g1 = tmem + CT::T_G1 + lane_base;
   const uint32_t t_gr = tmem + CT::T_GR + lane_base;
+  const uint32_t t_sn = tmem + CT::T_SN + lane_base;
   uint32_t phase = 0, phase_gr = 0;
   bool aborted = false;
   // bounded wait for the oldest commit on `bar` (or on `bar_gr`), decided by the whole CTA
@@ -199,6 +204,16 @@ __global__ void __launch_bounds__(ChunkTC::NT, 1) prefill_chunk_tc(const StepPar
     return any;
   };
   auto wait_mma = [&]() -> bool { return wait_on(&bar, phase); };
+  // a quarter (16 columns) of this warpgroup's half of the staged snapshot to
+  // the pool; the snapshot page is the same for the whole CTA
+  auto snap_piece = [&](int64_t page, int piece) {
+    if (page < 0) return;
+    float y[16];
+    tmem_ld16(t_sn + 64 * wg + 16 * piece, y);
+    float4* dst = reinterpret_cast<float4*>(pool + (page * p.HV + hv) * head + (int64_t)v * D + 64 * wg + 16 * piece);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) __stcs(dst + q, make_float4(y[4 * q], y[4 * q + 1], y[4 * q + 2], y[4 * q + 3]));
+  };
 
   const float expA = expf(p.A_log[hv]);
   const float dtb = p.dt_bias[hv];
@@ -294,8 +309,8 @@ __global__ void __launch_bounds__(ChunkTC::NT, 1) prefill_chunk_tc(const StepPar
       aborted = true;
       break;
     }
+    int64_t snap = -1;  // page receiving the chunk's initial state, staged in tensor memory
     {
-      int64_t snap = -1;
       if (c > 0) {
         const int64_t last = base - 1;  // last position of the previous chunk
         if (last >= pos_lo) snap = suffix_snapshot_page(p, u, static_cast<int>(last - pos_lo));
@@ -334,15 +349,13 @@ __global__ void __launch_bounds__(ChunkTC::NT, 1) prefill_chunk_tc(const StepPar
           x[1][i] = __uint_as_float(r1[i]);
         }
       }
+      if (snap >= 0) {
+        tmem_st32_issue(t_sn + 64 * wg, x[0]);
+        tmem_st32_issue(t_sn + 64 * wg + 32, x[1]);
+      }
 #pragma unroll
       for (int kk = 0; kk < 2; ++kk) {
         const int kc = 2 * wg + kk;
-        if (snap >= 0) {
-          float4* dst = reinterpret_cast<float4*>(pool + (snap * p.HV + hv) * head + (int64_t)v * D + 32 * kc);
-#pragma unroll
-          for (int q = 0; q < 8; ++q)
-            __stcs(dst + q, make_float4(x[kk][4 * q], x[kk][4 * q + 1], x[kk][4 * q + 2], x[kk][4 * q + 3]));
-        }
 #pragma unroll
         for (int q8 = 0; q8 < 4; ++q8) {
           uint32_t hw[4], lw[4];
@@ -382,6 +395,7 @@ __global__ void __launch_bounds__(ChunkTC::NT, 1) prefill_chunk_tc(const StepPar
       break;
     }
 
+    snap_piece(snap, 0);
     // ---- A and P rows from the Gram: thread (wg, r) takes columns 32 wg ..
     // 32 wg + 31 of row r (k row r < 64: A in fp32; q row r - 64: P as three
     // bf16 tiles, the B operand of the output product). A and K^T take space
@@ -436,6 +450,7 @@ __global__ void __launch_bounds__(ChunkTC::NT, 1) prefill_chunk_tc(const StepPar
       }
       ktw[tt] = make_uint4(w[0], w[1], w[2], w[3]);
     }
+    snap_piece(snap, 1);
     if (wait_mma()) {  // G1; also orders P before the reads below
       aborted = true;
       break;
@@ -465,6 +480,7 @@ __global__ void __launch_bounds__(ChunkTC::NT, 1) prefill_chunk_tc(const StepPar
       }
     }
     __syncthreads();
+    snap_piece(snap, 2);
     // ---- (I + A) U = R in two blocks of 32 tokens: each warpgroup takes 16
     // rows of the block for the part from the earlier block; the triangle
     // inside the block is finished by the first warpgroup, then by the second
@@ -525,6 +541,7 @@ __global__ void __launch_bounds__(ChunkTC::NT, 1) prefill_chunk_tc(const StepPar
         __syncthreads();
       }
     }
+    snap_piece(snap, 3);
     // ---- outputs o_t = e^{g_t} q^_t S0 + sum_{s<=t} P_ts U_s: U^T (three bf16
     // terms, replacing A) times P^T on the tensor cores (the six products of
     // the splits above the lowest order), then the state part added
