@@ -112,13 +112,20 @@ __device__ __forceinline__ void split3_bf16x8(const float* x, uint4& h, uint4& m
 
 // The token inputs of the chunk starting at absolute position `base` into
 // input buffer `buf`: k rows and q rows into the [K ; Q] operand tile, v rows
-// row-major; slots outside [pos_lo, pos_hi) are zero filled.
+// row-major; slots outside [pos_lo, pos_hi) are zero filled. Part `part` of
+// kLoadParts (one cp.async group each): the next chunk's copies are issued
+// in parts over the current chunk, because every CTA issuing its 48 KiB at
+// the same point stalled on the memory system.
+constexpr int kLoadParts = 4;
 __device__ __forceinline__ void chunk_issue_loads(const StepParams& p, unsigned char* sm, int buf, int64_t base,
-                                                  int64_t pos_lo, int64_t pos_hi, int64_t tok_lo, int h, int hv) {
+                                                  int64_t pos_lo, int64_t pos_hi, int64_t tok_lo, int h, int hv,
+                                                  int part) {
   using CT = ChunkTC;
   unsigned char* kq = sm + CT::KQ + buf * CT::KQ_BYTES;
   unsigned char* vv = sm + CT::VB + buf * CT::V_BYTES;
-  for (int id = threadIdx.x; id < 3 * CT::C * 16; id += CT::NT) {
+  constexpr int PER = 3 * CT::C * 16 / kLoadParts;
+  static_assert(PER % CT::NT == 0, "whole copies per thread and part");
+  for (int id = part * PER + threadIdx.x; id < (part + 1) * PER; id += CT::NT) {
     const int which = id / (CT::C * 16), rem = id % (CT::C * 16), j = rem / 16, piece = rem % 16;
     const int64_t pos = base + j;
     const bool valid = pos >= pos_lo && pos < pos_hi;
@@ -208,11 +215,27 @@ __global__ void __launch_bounds__(ChunkTC::NT, 1) prefill_chunk_tc(const StepPar
   // the pool; the snapshot page is the same for the whole CTA
   auto snap_piece = [&](int64_t page, int piece) {
     if (page < 0) return;
-    float y[16];
-    tmem_ld16(t_sn + 64 * wg + 16 * piece, y);
-    float4* dst = reinterpret_cast<float4*>(pool + (page * p.HV + hv) * head + (int64_t)v * D + 64 * wg + 16 * piece);
+    // 16x256b loads: in each 16-lane half of the warp's 32 lanes, four
+    // consecutive threads hold 8 consecutive columns of one lane (row), so
+    // each 8-byte store fills whole 32-byte sectors of the page row (the
+    // 32x32b shape gives each thread its own row: 16-byte pieces of 32
+    // rows per store instruction)
+    const int lane = tid & 31;
+    const uint32_t sp = static_cast<uint32_t>(32 * ((tid >> 5) & 3));
 #pragma unroll
-    for (int q = 0; q < 4; ++q) __stcs(dst + q, make_float4(y[4 * q], y[4 * q + 1], y[4 * q + 2], y[4 * q + 3]));
+    for (int half = 0; half < 2; ++half) {
+      uint32_t r[8];
+      tmem_ld16x256b_x2(tmem + CT::T_SN + ((sp + 16 * half) << 16) + 64 * wg + 16 * piece, r);
+#pragma unroll
+      for (int g = 0; g < 2; ++g)
+#pragma unroll
+        for (int hl = 0; hl < 2; ++hl) {
+          const int row = sp + 16 * half + 8 * hl + (lane >> 2);
+          const int col = 64 * wg + 16 * piece + 8 * g + 2 * (lane & 3);
+          __stcs(reinterpret_cast<float2*>(pool + (page * p.HV + hv) * head + (int64_t)row * D + col),
+                 make_float2(__uint_as_float(r[4 * g + 2 * hl]), __uint_as_float(r[4 * g + 2 * hl + 1])));
+        }
+    }
   };
 
   const float expA = expf(p.A_log[hv]);
@@ -228,8 +251,14 @@ __global__ void __launch_bounds__(ChunkTC::NT, 1) prefill_chunk_tc(const StepPar
       }
     }
   };
-  chunk_issue_loads(p, sm, 0, base0, pos_lo, pos_hi, u.tok0, h, hv);
+#pragma unroll 1
+  for (int part = 0; part < kLoadParts; ++part) chunk_issue_loads(p, sm, 0, base0, pos_lo, pos_hi, u.tok0, h, hv, part);
   load_ab(base0);
+  // part `part` of the next chunk's copies (they go to the other buffer,
+  // free since the previous chunk ended)
+  auto next_loads = [&](int c, int64_t base, int part) {
+    if (c + 1 < nchunks) chunk_issue_loads(p, sm, (c & 1) ^ 1, base + C, pos_lo, pos_hi, u.tok0, h, hv, part);
+  };
 
   for (int c = 0; c < nchunks && !aborted; ++c) {
     const int buf = c & 1;
@@ -250,10 +279,8 @@ __global__ void __launch_bounds__(ChunkTC::NT, 1) prefill_chunk_tc(const StepPar
         umma_bf16(tmem + CT::T_GR, umma_desc_add(dk, ks * 256), umma_desc_add(dk, ks * 256), id_gr, ks > 0);
       umma_commit(&bar_gr);
     }
-    if (c + 1 < nchunks) {
-      chunk_issue_loads(p, sm, buf ^ 1, base + C, pos_lo, pos_hi, u.tok0, h, hv);
-      load_ab(base + C);
-    }
+    next_loads(c, base, 0);
+    if (c + 1 < nchunks) load_ab(base + C);
     const unsigned char* kq = sm + CT::KQ + buf * CT::KQ_BYTES;
 
     // ---- per-token scalars: log alpha prefix (double), beta, norms
@@ -451,6 +478,7 @@ __global__ void __launch_bounds__(ChunkTC::NT, 1) prefill_chunk_tc(const StepPar
       ktw[tt] = make_uint4(w[0], w[1], w[2], w[3]);
     }
     snap_piece(snap, 1);
+    next_loads(c, base, 1);
     if (wait_mma()) {  // G1; also orders P before the reads below
       aborted = true;
       break;
@@ -481,6 +509,7 @@ __global__ void __launch_bounds__(ChunkTC::NT, 1) prefill_chunk_tc(const StepPar
     }
     __syncthreads();
     snap_piece(snap, 2);
+    next_loads(c, base, 2);
     // ---- (I + A) U = R in two blocks of 32 tokens: each warpgroup takes 16
     // rows of the block for the part from the earlier block; the triangle
     // inside the block is finished by the first warpgroup, then by the second
@@ -542,6 +571,7 @@ __global__ void __launch_bounds__(ChunkTC::NT, 1) prefill_chunk_tc(const StepPar
       }
     }
     snap_piece(snap, 3);
+    next_loads(c, base, 3);
     // ---- outputs o_t = e^{g_t} q^_t S0 + sum_{s<=t} P_ts U_s: U^T (three bf16
     // terms, replacing A) times P^T on the tensor cores (the six products of
     // the splits above the lowest order), then the state part added

@@ -119,6 +119,16 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float* x) {
 #pragma unroll
   for (int i = 0; i < 16; ++i) x[i] = __uint_as_float(r[i]);
 }
+// 16x256b shape, two 8-column groups: of the 16 lanes starting at the
+// address's lane, thread t of the warp holds lanes (t / 4) and (t / 4 + 8),
+// columns 2 (t % 4) and 2 (t % 4) + 1 of each group: r[4 g + 2 h + j] is
+// lane (t / 4 + 8 h), column 8 g + 2 (t % 4) + j.
+__device__ __forceinline__ void tmem_ld16x256b_x2(uint32_t taddr, uint32_t* r) {
+  asm volatile("tcgen05.ld.sync.aligned.16x256b.x2.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+               : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
 __device__ __forceinline__ void tmem_ld8(uint32_t taddr, float* x) {
   uint32_t r[8];
   asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
