@@ -172,12 +172,16 @@ __global__ void __launch_bounds__(KdaTC::NT, 1) kda_chunk_tc(const StepParams p)
 
   const float expA = expf(p.A_log[hv]);
   const float dtb = p.dt_bias[(int64_t)hv * D + v];
-  // the token inputs of chunk c into input buffer `buf` (zero past the run)
-  auto issue_loads = [&](int c, int buf) {
+  // the token inputs of chunk c into input buffer `buf` (zero past the run),
+  // part `part` of four (one cp.async group each): the next chunk's copies
+  // are spread over the current chunk rather than issued by every CTA at once
+  constexpr int kParts = 4, PER = 4 * C * 16 / kParts;
+  static_assert(PER % CT::NT == 0, "whole copies per thread and part");
+  auto issue_loads = [&](int c, int buf, int part) {
     unsigned char* raw = sm + CT::RAW + buf * CT::RAW_BYTES;
     const int nv = min(C, n - c * C);
     const int64_t t0 = u.tok0 + (int64_t)c * C;
-    for (int id = tid; id < 4 * C * 16; id += CT::NT) {
+    for (int id = part * PER + tid; id < (part + 1) * PER; id += CT::NT) {
       const int which = id / (C * 16), rem = id % (C * 16), j = rem / 16, piece = rem % 16;
       const bool valid = j < nv;
       const int64_t tok = t0 + j;
@@ -202,8 +206,12 @@ __global__ void __launch_bounds__(KdaTC::NT, 1) kda_chunk_tc(const StepParams p)
   // P past the diagonal (s > t) is never written by the pair loop: zero once
   for (int i = tid; i < 3 * CT::P_BYTES / 16; i += CT::NT)
     reinterpret_cast<uint4*>(sm + CT::P3)[i] = make_uint4(0u, 0u, 0u, 0u);
-  issue_loads(0, 0);
+#pragma unroll 1
+  for (int part = 0; part < kParts; ++part) issue_loads(0, 0, part);
   load_beta(0);
+  auto next_loads = [&](int c, int part) {
+    if (c + 1 < nchunks) issue_loads(c + 1, (c & 1) ^ 1, part);
+  };
 
   for (int c = 0; c < nchunks && !aborted; ++c) {
     const int buf = c & 1;
@@ -211,10 +219,8 @@ __global__ void __launch_bounds__(KdaTC::NT, 1) kda_chunk_tc(const StepParams p)
     const float cb = nb;
     cp_async_wait<0>();
     __syncthreads();
-    if (c + 1 < nchunks) {
-      issue_loads(c + 1, buf ^ 1);
-      load_beta(c + 1);
-    }
+    next_loads(c, 0);
+    if (c + 1 < nchunks) load_beta(c + 1);
     const unsigned char* raw = sm + CT::RAW + buf * CT::RAW_BYTES;
 
     // ---- prologue: norms (4 threads per k or q row), beta, the decay prefix
@@ -392,6 +398,7 @@ __global__ void __launch_bounds__(KdaTC::NT, 1) kda_chunk_tc(const StepParams p)
       umma_commit(&bar);
     }
 
+    next_loads(c, 1);
     // ---- A and P on the CUDA cores while G1 runs. The pairs (t, s <= t) of
     // row t come in groups of up to three consecutive s; group g goes to
     // thread g (187 groups), so the lanes of a warp share few t-rows and
@@ -485,6 +492,7 @@ __global__ void __launch_bounds__(KdaTC::NT, 1) kda_chunk_tc(const StepParams p)
       }
     }
     __syncthreads();
+    next_loads(c, 2);
     // ---- (I + A) U = R: the first warpgroup solves rows 0..15, then the
     // second subtracts what they contribute to rows 16..31 and solves those
     {
@@ -572,6 +580,7 @@ __global__ void __launch_bounds__(KdaTC::NT, 1) kda_chunk_tc(const StepParams p)
                       umma_desc_add(dk, j * CT::KBT_BYTES + ks * 256), id_up, true);
       umma_commit(&bar);
     }
+    next_loads(c, 3);
     if (wait_on(&bar_o, phase_o)) {
       aborted = true;
       break;
