@@ -282,11 +282,17 @@ step_stream_fp8(const StepParams p, int64_t n_tiles) {
             S[jj][e + 1] = y.y;
           }
         }
-        float m = 0.f;
+        // one partial maximum per row (independent chains), then their maximum
+        float mj[NR];
 #pragma unroll
-        for (int jj = 0; jj < NR; ++jj)
+        for (int jj = 0; jj < NR; ++jj) {
+          mj[jj] = 0.f;
 #pragma unroll
-          for (int e = 0; e < EPL; e += 2) m = absmax_acc2(m, S[jj][e], S[jj][e + 1]);
+          for (int e = 0; e < EPL; e += 2) mj[jj] = absmax_acc2(mj[jj], S[jj][e], S[jj][e + 1]);
+        }
+        float m = mj[0];
+#pragma unroll
+        for (int jj = 1; jj < NR; ++jj) m = fmaxf(m, mj[jj]);
         m = group_max<32>(m);
         if (lane == 0) s_amax[sub][warp] = m;
       }
