@@ -17,6 +17,7 @@
 #include "gdn_seq.cuh"
 #include "gdn_stream_fp8.cuh"
 #include "gdn_stream_i8.cuh"
+#include "gdn_group_i8.cuh"
 #include "gdn_chunk_tc.cuh"
 #include "gdn_kda_chunk.cuh"
 
@@ -195,7 +196,10 @@ int launch_one(StepParams p, int B, cudaStream_t s) {
   constexpr bool CODED = (SDT == ST_FP8 || SDT == ST_I8H);
   if constexpr (L == L_VFIRST && GATE == GATE_SCALAR) {
     if (p.T == 1) {
-      if constexpr (SDT == ST_I8H) return launch_pipe<StreamI8Shape<K>, step_stream_i8<K, IDX>>(p, B, s);
+      if constexpr (SDT == ST_I8H) {
+        if constexpr (K == 128) return launch_pipe<GroupI8Shape, step_group_i8<IDX>>(p, B, s);
+        else return launch_pipe<StreamI8Shape<K>, step_stream_i8<K, IDX>>(p, B, s);
+      }
       else if constexpr (SDT == ST_FP8) {
         if (p.V % 128 == 0) return launch_pipe<StreamFp8Shape<K, 2>, step_stream_fp8<K, IDX, 2>>(p, B, s);
         return launch_pipe<StreamFp8Shape<K, 1>, step_stream_fp8<K, IDX, 1>>(p, B, s);

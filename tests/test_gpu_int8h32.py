@@ -126,3 +126,15 @@ def test_int8h32_single_token_padded_stored_readout_k256():
                        indices=[3, -1, 99, 0, 5], readout="stored", index_dtype="i64")
     assert r["err"] == G.GDN_FLAG_SLOT_RANGE
     assert np.all(r["out"][[1, 2]] == 0)
+
+
+@pytest.mark.parametrize("in_dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("readout", ["working", "stored"])
+def test_int8h32_single_token_k128_group_kernel(in_dtype, readout):
+    """K = 128 single-token V_FIRST decode (one warp per scale group): both
+    readouts and input dtypes, a padded slot, an out-of-range slot, GQA, and
+    V = 256 (eight groups per head)."""
+    r = gdn_slots_case(103, B=6, T=1, H=2, HV=4, K=128, V=256, num_slots=8, state_dtype=I8, in_dtype=in_dtype,
+                       indices=[5, -1, 0, 11, 7, 2], readout=readout, index_dtype="i32")
+    assert r["err"] == G.GDN_FLAG_SLOT_RANGE
+    assert np.all(r["out"][[1, 3]] == 0)
