@@ -47,17 +47,23 @@ struct GroupI8Shape {
   static constexpr int NS = 3;                   // stages in the ring
   // one stage: codes | K scales | q row | k row | v slice (inputs sized for
   // fp32) | header: gate and beta words, A_log, dt_bias, status, unit index
-  // within the slot, write slot, change level, gate-index parity
+  // within the slot, write slot, change level, gate-index parity.
+  // Per-channel vectors that every lane reads in its 16-channel block (the
+  // scales, k, and later r' and s') are padded by 16 bytes per block, so that
+  // the 8 blocks of a row fall in distinct banks: block b starts at
+  // b (16 w + 16) for elements of w bytes (pad16_ofs).
   static constexpr int CODES = VT * K;
-  static constexpr int O_SC = CODES, O_Q = O_SC + K * 4, O_K = O_Q + K * 4, O_V = O_K + K * 4;
+  static constexpr int PADV = K * 4 + (K / EPL) * 16;   // a padded vector of fp32
+  static constexpr int O_SC = CODES, O_Q = O_SC + PADV, O_K = O_Q + K * 4, O_V = O_K + PADV;
   static constexpr int O_HDR = O_V + VT * 4;
   static constexpr int STAGE = O_HDR + 48;
   static constexpr int SMEM = NS * STAGE;        // dynamic shared memory
   // after pass 2 the stage's code area holds the partial maxima [RB][K], the
-  // new r' and (for a stored readout) the new s'
-  static constexpr int O_MX = 0, O_R = RB * K * 4, O_S = O_R + K * 4;
+  // new r' and (for a stored readout) the new s', all padded
+  static constexpr int O_MX = 0, O_R = RB * PADV, O_S = O_R + PADV;
   static constexpr int MIN_CTAS = 12;
-  static_assert(STAGE % 16 == 0 && O_S + K * 4 <= CODES, "stage layout");
+  static_assert(STAGE % 16 == 0 && O_S + PADV <= CODES, "stage layout");
+  static_assert(MIN_CTAS * (SMEM + 1024) <= 233472, "the ring of 12 warps fits one SM's shared memory");
   static_assert(NR == LPR, "the reduce-scatter of 2 NR sums over LPR lanes leaves one row's pair per lane");
 };
 
@@ -79,6 +85,10 @@ __device__ __forceinline__ float2 rs_row_pairs(float* x, int cc) {
     return rs_row_pairs<N / 2, O / 2>(x, cc);
   }
 }
+
+// Byte offset of 16-byte chunk c of a vector stored with a 16-byte pad after
+// every `cpb` chunks (one lane block of 16 channels).
+__device__ __forceinline__ int pad16_ofs(int c, int cpb) { return 16 * c + 16 * (c / cpb); }
 
 // 16 int8 codes (16 bytes) -> their values as floats
 __device__ __forceinline__ void decode_i8x16(uint4 raw, float* c) {
@@ -132,6 +142,8 @@ step_group_i8(const StepParams p, int64_t n_units) {
   const int n_my = static_cast<int>(u_end - u_begin);
   if (n_my <= 0) return;
   const int nqk = K * in_b / 16;       // 16-byte chunks of a q (or k) row
+  const int kblk = 16 * in_b + 16;     // a lane block of the padded k row (bytes)
+  constexpr int FBLK = EPL * 4 + 16;   // ... of a padded fp32 vector
   const int nvv = VT * in_b / 16;      // ... of the v slice
 
   // ---- producer side: copies of unit u_begin + i into stage i % NS
@@ -162,12 +174,12 @@ step_group_i8(const StepParams p, int64_t n_units) {
 #pragma unroll
       for (int r = 0; r < NR; ++r) cp_async16(st + my_off + r * ROWB, src + r * ROWB, true);
       const char* scb = reinterpret_cast<const char*>(p.scales + (pc_src * per_b + pc.within) * K);
-      cp_async16(st + PS::O_SC + lane * 16, scb + lane * 16, true);
+      cp_async16(st + PS::O_SC + pad16_ofs(lane, 4), scb + lane * 16, true);
       const int64_t qk_row = ((int64_t)pc.b * p.H + pc.h) * K * in_b;
       for (int c = lane; c < 2 * nqk; c += 32) {
         const bool isk = c >= nqk;
         const int ch = c - (isk ? nqk : 0);
-        cp_async16(st + (isk ? PS::O_K : PS::O_Q) + ch * 16,
+        cp_async16(st + (isk ? PS::O_K + pad16_ofs(ch, in_b) : PS::O_Q + ch * 16),
                    reinterpret_cast<const char*>(isk ? p.k : p.q) + qk_row + ch * 16, true);
       }
       if (lane < nvv)
@@ -229,7 +241,7 @@ step_group_i8(const StepParams p, int64_t n_units) {
     {
       float qv[EPL], kv[EPL], sv[EPL];
       ld_in_vec<EPL>(st + PS::O_Q, cc * EPL, in_bf16, qv);
-      ld_in_vec<EPL>(st + PS::O_K, cc * EPL, in_bf16, kv);
+      ld_in_vec<EPL>(st + PS::O_K + cc * kblk, 0, in_bf16, kv);
       if (change >= 2) {
         float2 sq = make_float2(0.f, 0.f), sk = sq, sqk = sq;
 #pragma unroll
@@ -250,7 +262,7 @@ step_group_i8(const StepParams p, int64_t n_units) {
         }
         qk = dqk * iq * ik;
       }
-      ld_vec16_f32(st + PS::O_SC + cc * EPL * 4, sv);
+      ld_vec16_f32(st + PS::O_SC + cc * FBLK, sv);
       // the scales ride on k and q for the dots
 #pragma unroll
       for (int e = 0; e < EPL; e += 2) {
@@ -300,15 +312,15 @@ step_group_i8(const StepParams p, int64_t n_units) {
     __syncwarp();
     {
       const float2 a2 = make_float2(alpha, alpha);
-      float4* mx = reinterpret_cast<float4*>(st + PS::O_MX + (rb * K + cc * EPL) * 4);
+      float4* mx = reinterpret_cast<float4*>(st + PS::O_MX + rb * PS::PADV + cc * FBLK);
 #pragma unroll
       for (int c4 = 0; c4 < EPL / 4; ++c4) {
         float m[4];
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
           const int e = 4 * c4 + 2 * h;
-          const float2 k2 = ld_in_pair(st + PS::O_K, cc * EPL + e, in_bf16);
-          const float2 f2 = __fmul2_rn(a2, *reinterpret_cast<const float2*>(st + PS::O_SC + (cc * EPL + e) * 4));
+          const float2 k2 = ld_in_pair(st + PS::O_K + cc * kblk, e, in_bf16);
+          const float2 f2 = __fmul2_rn(a2, *reinterpret_cast<const float2*>(st + PS::O_SC + cc * FBLK + e * 4));
 #pragma unroll
           for (int r = 0; r < NR; ++r) {
             const float2 y = __ffma2_rn(f2, make_float2(S[r][e], S[r][e + 1]),
@@ -332,11 +344,11 @@ step_group_i8(const StepParams p, int64_t n_units) {
     __syncwarp();
     {
       // lane l: key channels 4 l .. 4 l + 3
-      const float4* mx = reinterpret_cast<const float4*>(st + PS::O_MX);
-      float4 a = mx[lane];
+      const unsigned char* mx = st + PS::O_MX + pad16_ofs(lane, 4);
+      float4 a = *reinterpret_cast<const float4*>(mx);
 #pragma unroll
       for (int b = 1; b < PS::RB; ++b) {
-        const float4 t = mx[b * (K / 4) + lane];
+        const float4 t = *reinterpret_cast<const float4*>(mx + b * PS::PADV);
         a = make_float4(fmaxf(a.x, t.x), fmaxf(a.y, t.y), fmaxf(a.z, t.z), fmaxf(a.w, t.w));
       }
       float4 s4, r4;
@@ -347,8 +359,8 @@ step_group_i8(const StepParams p, int64_t n_units) {
       float* dsc = p.scales + (dst_slot * per_b + within) * K;
       st_stream16(dsc + 4 * lane, make_uint4(__float_as_uint(s4.x), __float_as_uint(s4.y), __float_as_uint(s4.z),
                                              __float_as_uint(s4.w)));
-      reinterpret_cast<float4*>(st + PS::O_R)[lane] = r4;
-      if (stored_readout) reinterpret_cast<float4*>(st + PS::O_S)[lane] = s4;
+      *reinterpret_cast<float4*>(st + PS::O_R + pad16_ofs(lane, 4)) = r4;
+      if (stored_readout) *reinterpret_cast<float4*>(st + PS::O_S + pad16_ofs(lane, 4)) = s4;
     }
     __syncwarp();
 
@@ -358,7 +370,7 @@ step_group_i8(const StepParams p, int64_t n_units) {
       uint32_t cw[NR][EPL / 4];
 #pragma unroll
       for (int c4 = 0; c4 < EPL / 4; ++c4) {
-        const float4 r4 = *reinterpret_cast<const float4*>(st + PS::O_R + (cc * EPL + 4 * c4) * 4);
+        const float4 r4 = *reinterpret_cast<const float4*>(st + PS::O_R + cc * FBLK + 16 * c4);
 #pragma unroll
         for (int r = 0; r < NR; ++r) {
           const float2 lo = __fmul2_rn(make_float2(S[r][4 * c4], S[r][4 * c4 + 1]), make_float2(r4.x, r4.y));
@@ -379,7 +391,7 @@ step_group_i8(const StepParams p, int64_t n_units) {
             float c[4], q4[4];
             i8x4_to_float(cw[r][c4], c);
             ld_in_vec<4>(st + PS::O_Q, cc * EPL + 4 * c4, in_bf16, q4);
-            const float4 s4 = *reinterpret_cast<const float4*>(st + PS::O_S + (cc * EPL + 4 * c4) * 4);
+            const float4 s4 = *reinterpret_cast<const float4*>(st + PS::O_S + cc * FBLK + 16 * c4);
             y = fmaf(q4[0] * s4.x, c[0], y);
             y = fmaf(q4[1] * s4.y, c[1], y);
             y = fmaf(q4[2] * s4.z, c[2], y);

@@ -181,14 +181,19 @@ def check_stored_readout(out_gpu, t, idx, pool_after, scales_after, units, layou
 def gdn_slots_case(seed, B, T, H, HV, K, V, num_slots, layout="V_FIRST", state_dtype="f32",
                    in_dtype="bf16", out_dtype="f32", index_dtype="i32", readout="working",
                    indices=None, use_qk_l2norm=True, scale=None, tokens=None, block_v=64,
-                   check=True, units=None):
-    """Run one GDN slot decode on the GPU and the oracle; assert parity. Returns a dict."""
+                   check=True, units=None, zero_slots=()):
+    """Run one GDN slot decode on the GPU and the oracle; assert parity. Returns a dict.
+    `zero_slots` start from an all-zero state (codes and scales)."""
     t = tokens or W.gdn_tokens(seed, B, T, H, HV, K, V, in_dtype)
     idx = np.asarray(indices if indices is not None else W.slot_indices(seed, B, num_slots), np.int64)
     live = [int(s) for s in idx if 0 <= s < num_slots]
     exact = set(live) if units is None else {int(idx[b]) for b, _ in units if 0 <= idx[b] < num_slots}
     pool, scales = W.device_pool(seed, num_slots, HV, K, V, layout, state_dtype, block_v,
                                  exact_slots=sorted(exact))
+    for zs in zero_slots:
+        pool[zs] = 0
+        if scales is not None:
+            scales[zs] = 0
     before = pool_host(pool)
     sc_before = scales.cpu().numpy() if scales is not None else None
     err = torch.zeros(1, dtype=torch.int32, device="cuda")

@@ -488,3 +488,21 @@ def test_paged_coded_many_tiles_per_cta(state_dtype):
     res = gdn_paged_case(33, B=B, H=16, HV=HV, K=128, V=128, page_size=64, max_len=256, n_share=8,
                          share_pages=2, force_lens={0: 129, 1: 129}, state_dtype=state_dtype, units=units)
     assert res["err"] == 0
+
+
+@pytest.mark.parametrize("in_dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("readout", ["working", "stored"])
+def test_fp8_single_token_k128_readouts_zero_tile(in_dtype, readout):
+    """K = 128 single-token fp8 decode (the streaming kernel): both readouts
+    and input dtypes, GQA, V = 256 (two units of two tiles per head), a padded
+    and an out-of-range slot, and a sequence whose state and v are zero, so
+    that its tiles stay zero (scale 0, +0 codes)."""
+    B, H, HV, K, V = 6, 2, 4, 128, 256
+    t = W.gdn_tokens(31, B, 1, H, HV, K, V, in_dtype)
+    t["v"][4] = 0.0
+    r = gdn_slots_case(31, B=B, T=1, H=H, HV=HV, K=K, V=V, num_slots=8, state_dtype="fp8_e4m3",
+                       in_dtype=in_dtype, indices=[5, -1, 0, 11, 7, 2], readout=readout, tokens=t,
+                       zero_slots=[7])
+    assert r["err"] == G.GDN_FLAG_SLOT_RANGE
+    assert np.all(r["out"][[1, 3]] == 0)
+    assert not r["pool_after"][7].any() and not r["scales_after"][7].any()

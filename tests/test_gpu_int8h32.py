@@ -132,9 +132,14 @@ def test_int8h32_single_token_padded_stored_readout_k256():
 @pytest.mark.parametrize("readout", ["working", "stored"])
 def test_int8h32_single_token_k128_group_kernel(in_dtype, readout):
     """K = 128 single-token V_FIRST decode (one warp per scale group): both
-    readouts and input dtypes, a padded slot, an out-of-range slot, GQA, and
-    V = 256 (eight groups per head)."""
+    readouts and input dtypes, a padded slot, an out-of-range slot, GQA,
+    V = 256 (eight groups per head), and a sequence whose state and v are
+    zero, so that its groups stay zero (scales 0, codes 0)."""
+    t = W.gdn_tokens(103, 6, 1, 2, 4, 128, 256, in_dtype)
+    t["v"][4] = 0.0
     r = gdn_slots_case(103, B=6, T=1, H=2, HV=4, K=128, V=256, num_slots=8, state_dtype=I8, in_dtype=in_dtype,
-                       indices=[5, -1, 0, 11, 7, 2], readout=readout, index_dtype="i32")
+                       indices=[5, -1, 0, 11, 7, 2], readout=readout, index_dtype="i32", tokens=t,
+                       zero_slots=[7])
     assert r["err"] == G.GDN_FLAG_SLOT_RANGE
     assert np.all(r["out"][[1, 3]] == 0)
+    assert not r["pool_after"][7].any() and not r["scales_after"][7].any()
