@@ -105,9 +105,16 @@ step_seq(const StepParams p) {
   static_assert(!I8 || VC % 32 == 0, "whole scale groups per tile");
   static_assert(!I8 || !VF || 32 % (NR * RPW) == 0, "a warp's rows stay inside one scale group");
 
+  // K_FIRST fp32 with a decay per key channel (KDA): a thread reads one key
+  // row at a time, so the row's scalars sit in pairs, (alpha k^, alpha q^)
+  // for the dots and (k^, alpha) for the update, one 8-byte load each (s_q
+  // keeps q^ for a stored readout)
+  constexpr bool KW = !VF && GATE == GATE_VECTOR && SDT == ST_F32;
   __shared__ __align__(16) float s_q[TC][K];
-  __shared__ __align__(16) float s_k[TC][K];
-  __shared__ __align__(16) float s_a[TC][GATE == GATE_VECTOR ? K : 1];
+  __shared__ __align__(16) float s_k[TC][KW ? 1 : K];
+  __shared__ __align__(16) float s_a[TC][(GATE == GATE_VECTOR && !KW) ? K : 1];
+  __shared__ __align__(16) float2 s_wd[KW ? TC : 1][KW ? K : 1];
+  __shared__ __align__(16) float2 s_wu[KW ? TC : 1][KW ? K : 1];
   __shared__ __align__(16) float s_v[TC][VC];
   __shared__ float s_b[TC], s_qk[TC];
   __shared__ float s_amax[2][NW];
@@ -282,17 +289,31 @@ step_seq(const StepParams p) {
         iq *= rsqrtf(sq + kL2Eps);
         ik = rsqrtf(sk + kL2Eps);
       }
-#pragma unroll
-      for (int e = 0; e < KPL; ++e) {
-        s_q[tt][lane * KPL + e] = qn[e] * iq;
-        s_k[tt][lane * KPL + e] = kn[e] * ik;
-      }
-      if constexpr (GATE == GATE_VECTOR) {
+      if constexpr (KW) {
         float gv[KPL], db[KPL];
         ld_in_vec<KPL>(p.gate, ((int64_t)tok * p.HV + hv) * K + lane * KPL, in_bf16, gv);
         ld_in_vec<KPL>(p.dt_bias, (int64_t)hv * K + lane * KPL, false, db);
 #pragma unroll
-        for (int e = 0; e < KPL; ++e) s_a[tt][lane * KPL + e] = decay_of(expA, gv[e] + db[e]);
+        for (int e = 0; e < KPL; ++e) {
+          const float a = decay_of(expA, gv[e] + db[e]);
+          const float kh = kn[e] * ik, qh = qn[e] * iq;
+          s_q[tt][lane * KPL + e] = qh;
+          s_wd[tt][lane * KPL + e] = make_float2(a * kh, a * qh);
+          s_wu[tt][lane * KPL + e] = make_float2(kh, a);
+        }
+      } else {
+#pragma unroll
+        for (int e = 0; e < KPL; ++e) {
+          s_q[tt][lane * KPL + e] = qn[e] * iq;
+          s_k[tt][lane * KPL + e] = kn[e] * ik;
+        }
+        if constexpr (GATE == GATE_VECTOR) {
+          float gv[KPL], db[KPL];
+          ld_in_vec<KPL>(p.gate, ((int64_t)tok * p.HV + hv) * K + lane * KPL, in_bf16, gv);
+          ld_in_vec<KPL>(p.dt_bias, (int64_t)hv * K + lane * KPL, false, db);
+#pragma unroll
+          for (int e = 0; e < KPL; ++e) s_a[tt][lane * KPL + e] = decay_of(expA, gv[e] + db[e]);
+        }
       }
       for (int c = lane; c < VC; c += 32) {
         float x = ld_in1(p.v, ((int64_t)tok * p.HV + hv) * V + v0 + c, in_bf16);
@@ -349,12 +370,20 @@ step_seq(const StepParams p) {
 #pragma unroll
         for (int jj = 0; jj < NR; ++jj) {
           const int r = g + RG * jj;
-          kw[jj] = s_k[tt][r];
-          float wk = kw[jj], wq = s_q[tt][r];
-          if constexpr (GATE == GATE_VECTOR) {
-            const float a = s_a[tt][r];
-            wk *= a;
-            wq *= a;
+          float wk, wq;
+          if constexpr (KW) {
+            const float2 w = s_wd[tt][r];
+            wk = w.x;
+            wq = w.y;
+          } else {
+            kw[jj] = s_k[tt][r];
+            wk = kw[jj];
+            wq = s_q[tt][r];
+            if constexpr (GATE == GATE_VECTOR) {
+              const float a = s_a[tt][r];
+              wk *= a;
+              wq *= a;
+            }
           }
           const float2 wk2 = make_float2(wk, wk), wq2 = make_float2(wq, wq);
 #pragma unroll
@@ -409,12 +438,18 @@ step_seq(const StepParams p) {
             if constexpr (GATE == GATE_SCALAR) f2 = make_float2(alpha, alpha);
             else f2 = make_float2(s_a[tt][kofs + e], s_a[tt][kofs + e + 1]);
           } else {
-            k2 = make_float2(kw[jj], kw[jj]);
             u2 = make_float2(uu[e], uu[e + 1]);
-            if constexpr (GATE == GATE_SCALAR) f2 = make_float2(alpha, alpha);
-            else {
-              const float a = s_a[tt][g + RG * jj];
-              f2 = make_float2(a, a);
+            if constexpr (KW) {
+              const float2 w = s_wu[tt][g + RG * jj];
+              k2 = make_float2(w.x, w.x);
+              f2 = make_float2(w.y, w.y);
+            } else {
+              k2 = make_float2(kw[jj], kw[jj]);
+              if constexpr (GATE == GATE_SCALAR) f2 = make_float2(alpha, alpha);
+              else {
+                const float a = s_a[tt][g + RG * jj];
+                f2 = make_float2(a, a);
+              }
             }
           }
           const float2 y = __ffma2_rn(k2, u2, __fmul2_rn(f2, make_float2(S[jj][e], S[jj][e + 1])));

@@ -143,3 +143,20 @@ def test_int8h32_single_token_k128_group_kernel(in_dtype, readout):
     assert r["err"] == G.GDN_FLAG_SLOT_RANGE
     assert np.all(r["out"][[1, 3]] == 0)
     assert not r["pool_after"][7].any() and not r["scales_after"][7].any()
+
+
+def test_int8h32_many_groups_per_warp_with_padding():
+    """Enough groups that every warp of the K = 128 kernel streams dozens of
+    them across sequence boundaries, with padded and out-of-range sequences
+    among them and four value heads per key head; checked on a sample of
+    (sequence, head) pairs and on the padded rows."""
+    B, H, HV, K, V, num_slots = 256, 8, 32, 128, 128, 260
+    idx = np.random.default_rng(104).permutation(num_slots)[:B].astype(np.int64)
+    idx[::7] = -1
+    idx[5] = num_slots + 3
+    r = np.random.default_rng(105)
+    units = sorted({(int(b), int(h)) for b, h in zip(r.integers(0, B, 300), r.integers(0, HV, 300))})
+    units += [(b, h) for b in (0, 4, 6, 8) for h in (0, HV - 1)]
+    res = gdn_slots_case(104, B, 1, H, HV, K, V, num_slots, state_dtype=I8, indices=idx, units=sorted(set(units)))
+    assert res["err"] == G.GDN_FLAG_SLOT_RANGE
+    assert np.all(res["out"][idx < 0] == 0) and np.all(res["out"][5] == 0)
