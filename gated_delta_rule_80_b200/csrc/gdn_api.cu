@@ -216,7 +216,9 @@ int launch_one(StepParams p, int B, cudaStream_t s) {
       return launch_seq_nw<L, SDT, K, GATE, IDX, 4>(p, B, s);
     }
   } else {
-    return launch_seq_nw<L, SDT, K, GATE, IDX, (CODED && K == 256) ? 8 : 4>(p, B, s);
+    // eight warps for wide int8/fp8 rows, and for fp32 K = 32 (one row per
+    // thread: the shortest per-token chain for the latency-bound small heads)
+    return launch_seq_nw<L, SDT, K, GATE, IDX, ((CODED && K == 256) || (SDT == ST_F32 && K == 32)) ? 8 : 4>(p, B, s);
   }
 }
 

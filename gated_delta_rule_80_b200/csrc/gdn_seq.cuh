@@ -59,8 +59,9 @@ struct ReduceScatterS {
 template <int SDT, int LAYOUT, int K, int NW>
 struct SeqShape {
   // tokens per prologue chunk (4 for int8 K=256, whose scale-group buffers
-  // would otherwise push the static shared memory past 48 KiB)
-  static constexpr int TC = (SDT == ST_I8H && K == 256) ? 4 : 8;
+  // would otherwise push the static shared memory past 48 KiB; 16 for small
+  // heads, whose runs are latency-bound and whose buffers are small)
+  static constexpr int TC = (SDT == ST_I8H && K == 256) ? 4 : (K <= 64 ? 16 : 8);
   // V_FIRST: 16-byte vectors (32 for a K=256 fp32 row, so that it fits a warp)
   static constexpr int VB_V = (SDT == ST_F32 && K == 256) ? 32 : 16;
   // K_FIRST: 4 elements per lane, CPL lanes per row segment (16 columns per
