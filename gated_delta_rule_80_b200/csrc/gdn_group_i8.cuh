@@ -12,7 +12,7 @@
 // Lane l = 8 rb + cc holds rows 8 rb .. 8 rb + 7 of the group and key
 // channels 16 cc .. 16 cc + 15 of each (128 state values):
 //   - the amax of a key channel runs over the group's 32 rows, i.e. over the
-//     lane's own 8 rows and the 4 lanes of the same cc (through a 2 KiB
+//     lane's own 8 rows and the 4 lanes of the same cc (through a 2.5 KiB
 //     buffer in the consumed stage);
 //   - the dot products k.S and q.S of a row run over the 8 lanes of the same
 //     rb; their reduce-scatter leaves row l's pair on lane l, which is where
