@@ -197,7 +197,13 @@ int launch_one(StepParams p, int B, cudaStream_t s) {
   if constexpr (L == L_VFIRST && GATE == GATE_SCALAR) {
     if (p.T == 1) {
       if constexpr (SDT == ST_I8H) {
-        if constexpr (K == 128) return launch_pipe<GroupI8Shape, step_group_i8<IDX>>(p, B, s);
+        if constexpr (K == 128) {
+          const bool bf = (p.flags & F_IN_BF16) != 0, st = (p.flags & F_READOUT_STORED) != 0;
+          if (bf) return st ? launch_pipe<GroupI8Shape, step_group_i8<IDX, true, true>>(p, B, s)
+                            : launch_pipe<GroupI8Shape, step_group_i8<IDX, true, false>>(p, B, s);
+          return st ? launch_pipe<GroupI8Shape, step_group_i8<IDX, false, true>>(p, B, s)
+                    : launch_pipe<GroupI8Shape, step_group_i8<IDX, false, false>>(p, B, s);
+        }
         else return launch_pipe<StreamI8Shape<K>, step_stream_i8<K, IDX>>(p, B, s);
       }
       else if constexpr (SDT == ST_FP8) {

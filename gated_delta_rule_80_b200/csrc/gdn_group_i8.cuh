@@ -115,7 +115,10 @@ __device__ __forceinline__ float2 ld_in_pair(const unsigned char* base, int i, b
   return *reinterpret_cast<const float2*>(base + 4 * i);
 }
 
-template <int IDX>
+// IN_BF16: bf16 token inputs (else fp32); STORED: the output is read from the
+// stored state (else from the working state). Both are fixed per call, so
+// they are template parameters and the unrolled loops carry no test of them.
+template <int IDX, bool IN_BF16, bool STORED>
 __global__ void __launch_bounds__(GroupI8Shape::NT, GroupI8Shape::MIN_CTAS)
 step_group_i8(const StepParams p, int64_t n_units) {
   using PS = GroupI8Shape;
@@ -130,10 +133,10 @@ step_group_i8(const StepParams p, int64_t n_units) {
   const int rb = lane / PS::LPR;
   const int row0 = rb * NR;            // the lane's first row; its rows are row0 .. row0 + NR - 1
   const int my_off = row0 * ROWB + cc * EPL;
-  const bool in_bf16 = (p.flags & F_IN_BF16) != 0;
+  constexpr bool in_bf16 = IN_BF16;
   const bool out_bf16 = (p.flags & F_OUT_BF16) != 0;
-  const bool stored_readout = (p.flags & F_READOUT_STORED) != 0;
-  const int in_b = in_bf16 ? 2 : 4;
+  constexpr bool stored_readout = STORED;
+  constexpr int in_b = in_bf16 ? 2 : 4;
   const int NVG = p.V / VT;
   const int64_t per_b = (int64_t)p.HV * NVG;        // groups of one sequence
   const int64_t slot_bytes = per_b * UNITB;         // one slot (or page) of the pool
