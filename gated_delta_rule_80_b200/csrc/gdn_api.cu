@@ -207,6 +207,18 @@ int launch_one(StepParams p, int B, cudaStream_t s) {
         else return launch_pipe<StreamI8Shape<K>, step_stream_i8<K, IDX>>(p, B, s);
       }
       else if constexpr (SDT == ST_FP8) {
+        if constexpr (K == 128) {
+          // the configured width: input dtype and readout fixed per instantiation
+          if (p.V % 128 == 0) {
+            const int fl = ((p.flags & F_IN_BF16) ? 1 : 0) | ((p.flags & F_READOUT_STORED) ? 2 : 0);
+            switch (fl) {
+              case 0: return launch_pipe<StreamFp8Shape<K, 2>, step_stream_fp8<K, IDX, 2, 0>>(p, B, s);
+              case 1: return launch_pipe<StreamFp8Shape<K, 2>, step_stream_fp8<K, IDX, 2, 1>>(p, B, s);
+              case 2: return launch_pipe<StreamFp8Shape<K, 2>, step_stream_fp8<K, IDX, 2, 2>>(p, B, s);
+              default: return launch_pipe<StreamFp8Shape<K, 2>, step_stream_fp8<K, IDX, 2, 3>>(p, B, s);
+            }
+          }
+        }
         if (p.V % 128 == 0) return launch_pipe<StreamFp8Shape<K, 2>, step_stream_fp8<K, IDX, 2>>(p, B, s);
         return launch_pipe<StreamFp8Shape<K, 1>, step_stream_fp8<K, IDX, 1>>(p, B, s);
       }

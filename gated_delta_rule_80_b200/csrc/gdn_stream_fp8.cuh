@@ -57,7 +57,10 @@ struct StreamFp8Shape {
   static_assert(STAGE % 16 == 0, "16-byte chunks");
 };
 
-template <int K, int IDX, int TPU>
+// FL: the call's input dtype and readout fixed at compile time (bit 0: bf16
+// inputs, bit 1: stored readout), so that the unrolled loops carry no test of
+// them; -1 reads both from the flags at run time.
+template <int K, int IDX, int TPU, int FL = -1>
 __global__ void __launch_bounds__(StreamFp8Shape<K, TPU>::NT, StreamFp8Shape<K, TPU>::MIN_CTAS)
 step_stream_fp8(const StepParams p, int64_t n_tiles) {
   using PS = StreamFp8Shape<K, TPU>;
@@ -89,9 +92,9 @@ step_stream_fp8(const StepParams p, int64_t n_tiles) {
   const int row0r = warp * NR * RPW + ri;  // tile row of row jj: row0r + jj * RPW
   const int myrow_t = row0r + myrow * RPW;
   const int my_off = row0r * ROWB + kofs;  // this thread's first chunk in a tile
-  const bool in_bf16 = (p.flags & F_IN_BF16) != 0;
+  const bool in_bf16 = FL < 0 ? (p.flags & F_IN_BF16) != 0 : (FL & 1) != 0;
   const bool out_bf16 = (p.flags & F_OUT_BF16) != 0;
-  const bool stored_readout = (p.flags & F_READOUT_STORED) != 0;
+  const bool stored_readout = FL < 0 ? (p.flags & F_READOUT_STORED) != 0 : (FL & 2) != 0;
   const int in_b = in_bf16 ? 2 : 4;
   const int NVT = p.V / VT;
   const int64_t per_b = (int64_t)p.HV * NVT;        // units of one sequence
