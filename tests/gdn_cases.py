@@ -284,6 +284,12 @@ def gdn_paged_case(seed, B, H, HV, K, V, page_size, max_len, n_share, share_page
     pos = {pg: i for i, pg in enumerate(write_pages)}
     sub_writes = {(pos[pg], hv): w for (pg, hv), w in writes.items()}
     res["state_err"] = check_state(after_w, sc_after_w, sub_writes, state_dtype, layout)
+    if state_dtype in CODED and readout == "stored" and T == 1:
+        # the conditional check: o is q^ times the state the kernel stored in
+        # the sequence's write page
+        dst = np.array([pos.get(int(rows[bb, 1]), -1) for bb in range(B)])
+        check_stored_readout(out_h, t, dst, after_w, sc_after_w, todo, layout, None, True, len(write_pages),
+                             64, state_dtype)
     keep = torch.ones(pt.num_pages, dtype=torch.bool, device="cuda")
     keep[wp] = False
     assert torch.equal(pool[keep], snap[keep]), "a page that is not a write page changed"

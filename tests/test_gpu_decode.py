@@ -506,3 +506,12 @@ def test_fp8_single_token_k128_readouts_zero_tile(in_dtype, readout):
     assert r["err"] == G.GDN_FLAG_SLOT_RANGE
     assert np.all(r["out"][[1, 3]] == 0)
     assert not r["pool_after"][7].any() and not r["scales_after"][7].any()
+
+
+@pytest.mark.parametrize("readout", ["working", "stored"])
+def test_fp8_k128_paged_single_token(readout):
+    """K = 128 single-token fp8 decode on a paged pool (copy-on-new-page for
+    the sequences whose last page is new), both readouts; the stored readout
+    is also held at 1e-4 to q^ times the state written to the page."""
+    gdn_paged_case(32, B=6, H=1, HV=2, K=128, V=128, page_size=8, max_len=60, n_share=2, share_pages=2,
+                   force_lens={0: 17, 1: 9}, state_dtype="fp8_e4m3", readout=readout)

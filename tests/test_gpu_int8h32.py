@@ -160,3 +160,19 @@ def test_int8h32_many_groups_per_warp_with_padding():
     res = gdn_slots_case(104, B, 1, H, HV, K, V, num_slots, state_dtype=I8, indices=idx, units=sorted(set(units)))
     assert res["err"] == G.GDN_FLAG_SLOT_RANGE
     assert np.all(res["out"][idx < 0] == 0) and np.all(res["out"][5] == 0)
+
+
+def test_int8h32_k128_no_l2norm_custom_scale():
+    """K = 128 single-token decode without the q/k L2 norm and with a custom
+    q scale (the norms and the scale enter the group kernel only through the
+    reduced dots)."""
+    gdn_slots_case(106, B=5, T=1, H=2, HV=4, K=128, V=128, num_slots=7, state_dtype=I8, in_dtype="f32",
+                   use_qk_l2norm=False, scale=0.3)
+
+
+@pytest.mark.parametrize("readout", ["working", "stored"])
+def test_int8h32_k128_paged_single_token(readout):
+    """K = 128 single-token decode on a paged pool (copy-on-new-page for the
+    sequences whose last page is new) through the group kernel, both readouts."""
+    gdn_paged_case(107, B=6, H=1, HV=2, K=128, V=128, page_size=8, max_len=60, n_share=2, share_pages=2,
+                   force_lens={0: 17, 1: 9}, state_dtype=I8, readout=readout)
